@@ -1,0 +1,122 @@
+"""fp64 CPU oracle for the selective scan (S6) -- TEST INFRASTRUCTURE ONLY.
+
+Only the tests, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline /
+reference legs may import this package.  It shares no code with the CUDA
+library in ``selective_state_space_50_b200`` and never touches a GPU.
+
+The arithmetic lives in ``ssm_oracle.c`` (plain sequential C in double
+precision, OpenMP over (batch, channel) pairs); this module compiles it with
+gcc and wraps it with ctypes over numpy float64 arrays.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Dict, Optional
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "ssm_oracle.c")
+_LIB = os.path.join(_HERE, "libssm_oracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compiles ssm_oracle.c into libssm_oracle.so (gcc, -O2, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fno-fast-math", "-fopenmp", "-fPIC",
+                               "-shared", _SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        dp = ctypes.c_void_p
+        i = ctypes.c_int
+        lib.ssm_oracle_fwd.argtypes = [i, i, i, i] + [dp] * 8 + [i, i, dp, dp, dp, i]
+        lib.ssm_oracle_fwd.restype = i
+        lib.ssm_oracle_bwd.argtypes = [i, i, i, i] + [dp] * 8 + [i] + [dp] * 9 + [i]
+        lib.ssm_oracle_bwd.restype = i
+        lib.ssm_oracle_max_threads.restype = i
+        _lib = lib
+    return _lib
+
+
+def _p(x: Optional[np.ndarray]):
+    if x is None:
+        return None
+    assert x.dtype == np.float64 and x.flags.c_contiguous
+    return x.ctypes.data
+
+
+def _f64(x):
+    return None if x is None else np.ascontiguousarray(x, dtype=np.float64)
+
+
+def max_threads() -> int:
+    return int(_load().ssm_oracle_max_threads())
+
+
+def fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True,
+        zoh=False, h0=None, nthreads: int = 0):
+    """Returns (out [b,d,L], last_state [b,d,N]) in float64."""
+    u, delta, A, B, C = map(_f64, (u, delta, A, B, C))
+    D, z, delta_bias, h0 = map(_f64, (D, z, delta_bias, h0))
+    batch, dim, L = u.shape
+    N = A.shape[1]
+    assert delta.shape == u.shape and A.shape == (dim, N)
+    assert B.shape == (batch, N, L) and C.shape == (batch, N, L)
+    out = np.empty_like(u)
+    last = np.empty((batch, dim, N))
+    rc = _load().ssm_oracle_fwd(batch, dim, L, N, _p(u), _p(delta), _p(A), _p(B), _p(C),
+                                _p(D), _p(z), _p(delta_bias), int(bool(delta_softplus)),
+                                int(bool(zoh)), _p(h0), _p(out), _p(last), int(nthreads))
+    assert rc == 0
+    return out, last
+
+
+def bwd(u, delta, A, B, C, D, z, delta_bias, delta_softplus, dout,
+        nthreads: int = 0) -> Dict[str, np.ndarray]:
+    """Returns a dict of float64 gradients: du, ddelta, dA, dB, dC and, where the
+    matching input is given, dD, dz, ddelta_bias."""
+    u, delta, A, B, C, dout = map(_f64, (u, delta, A, B, C, dout))
+    D, z, delta_bias = map(_f64, (D, z, delta_bias))
+    batch, dim, L = u.shape
+    N = A.shape[1]
+    g = {"du": np.empty_like(u), "ddelta": np.empty_like(u), "dA": np.empty((dim, N)),
+         "dB": np.empty((batch, N, L)), "dC": np.empty((batch, N, L))}
+    g["dD"] = np.empty(dim) if D is not None else None
+    g["dz"] = np.empty_like(u) if z is not None else None
+    g["ddelta_bias"] = np.empty(dim) if delta_bias is not None else None
+    rc = _load().ssm_oracle_bwd(batch, dim, L, N, _p(u), _p(delta), _p(A), _p(B), _p(C),
+                                _p(D), _p(z), _p(delta_bias), int(bool(delta_softplus)),
+                                _p(dout), _p(g["du"]), _p(g["ddelta"]), _p(g["dA"]),
+                                _p(g["dB"]), _p(g["dC"]), _p(g["dD"]), _p(g["dz"]),
+                                _p(g["ddelta_bias"]), int(nthreads))
+    if rc != 0:
+        raise MemoryError("oracle bwd: allocation failed")
+    return {k: v for k, v in g.items() if v is not None}
+
+
+def fwd_workload(inputs: Dict[str, np.ndarray], w, nthreads: int = 0):
+    """Runs fwd on the fp64 values of a generated workload dict."""
+    return fwd(inputs["u_f64"], inputs["delta_f64"], inputs["A_f64"], inputs["B_f64"],
+               inputs["C_f64"], inputs["D_f64"] if w.has_D else None,
+               inputs["z_f64"] if w.has_z else None,
+               inputs["delta_bias_f64"] if w.has_bias else None, w.softplus,
+               nthreads=nthreads)
+
+
+def bwd_workload(inputs: Dict[str, np.ndarray], w, nthreads: int = 0):
+    return bwd(inputs["u_f64"], inputs["delta_f64"], inputs["A_f64"], inputs["B_f64"],
+               inputs["C_f64"], inputs["D_f64"] if w.has_D else None,
+               inputs["z_f64"] if w.has_z else None,
+               inputs["delta_bias_f64"] if w.has_bias else None, w.softplus,
+               inputs["dout_f64"], nthreads=nthreads)
