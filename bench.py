@@ -1,0 +1,360 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 selective-scan (S6) forward at the Mamba-130M layer
+shape (batch 8, seqlen 2048, dim 1536, dstate 16, bf16 io, fp32 state).
+
+One step = one forward selective scan over one batch of synthetic inputs (the
+whole hot path: softplus, discretisation, recurrence, readout, D skip and
+gate, fused in one kernel).  Prints one JSON line.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Timing: inputs are resident in HBM; each step is bracketed by CUDA events on
+the launching stream, and the L2 is flushed (a 256 MiB write) between steps,
+outside the events.  The device time of the K steps is summed; under torchrun
+every rank runs its own batch (weak scaling, no data-path collective) and
+rank 0 reports the max over ranks.  `e2e` repeats the measurement through the
+public binding with inputs copied from pinned host memory and the output
+copied back inside each timed step.  `--impl reference` times the fp64 CPU
+oracle on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "mamba130m_layer"
+METRIC = "selective-scan fwd B*L*D*N elems/s"
+UNIT = "elem/s"
+SM_COUNT_B200 = 148
+MUFU_EX2_PER_CLK_PER_SM = 16   # SFU ex2 throughput per SM per clock
+FALLBACK_HBM_GBS = 6650.0
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return {"hbm_gbs": FALLBACK_HBM_GBS, "sm_max_mhz": 1965.0}, "fallback"
+
+
+def algorithmic_bytes(w, io_bytes, with_last_state=True):
+    e = w.batch * w.dim * w.seqlen
+    n = e * io_bytes * (3 + 1)                          # u, delta, z in; out
+    n += 2 * w.batch * w.dstate * w.seqlen * io_bytes   # B, C
+    n += w.dim * w.dstate * 4 + 2 * w.dim * 4           # A, D, bias
+    if with_last_state:
+        n += w.batch * w.dim * w.dstate * 4
+    return n
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, index: int, period_s: float = 0.01):
+        self.index, self.period = index, period_s
+        self.samples, self.reasons = [], 0
+        self._stop = threading.Event()
+        self._th = None
+        self.max_mhz = None
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nv = None
+            return self
+
+        def run():
+            while not self._stop.is_set():
+                try:
+                    self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
+                    self.reasons |= self._nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                except Exception:
+                    pass
+                time.sleep(self.period)
+        self._th = threading.Thread(target=run, daemon=True)
+        self._th.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._th:
+            self._th.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        names = [v for k, v in self.REASONS.items() if self.reasons & k and v != "gpu_idle"]
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64,
+                     device="cuda" if dist.get_backend() == "nccl" else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def cpu_oracle_rate(w, inp, budget_s: float, nthreads: int = 0):
+    """Times the fp64 oracle on whole-batch channel slices until about
+    `budget_s` seconds of wall time are spent.  Returns (elem/s, threads, desc)."""
+    import oracle
+    nthreads = nthreads or oracle.max_threads()
+    # slices of 16 channels, all batch rows, full sequence
+    step = 16
+    done_elems, t_total, slices = 0, 0.0, 0
+    d0 = 0
+    while t_total < budget_s:
+        sl = slice(d0, d0 + step)
+        sub = {k: (v[:, sl] if k.split("_f64")[0] in ("u", "delta", "z") else
+                   v[sl] if k.split("_f64")[0] in ("A", "D", "delta_bias") else v)
+               for k, v in inp.items() if k.endswith("_f64")}
+        sub = {k: np.ascontiguousarray(v) for k, v in sub.items()}
+        t = time.perf_counter()
+        oracle.fwd(sub["u_f64"], sub["delta_f64"], sub["A_f64"], sub["B_f64"], sub["C_f64"],
+                   sub["D_f64"], sub["z_f64"], sub["delta_bias_f64"], w.softplus,
+                   nthreads=nthreads)
+        t_total += time.perf_counter() - t
+        done_elems += w.batch * step * w.seqlen
+        slices += 1
+        d0 = (d0 + step) % w.dim
+    desc = (f"{slices} slices of {step} channels x batch {w.batch} x seqlen {w.seqlen} "
+            f"({done_elems * w.dstate / 1e9:.3f} G state-steps) of the {w.name} forward, "
+            f"fp64, {t_total:.1f} s")
+    return done_elems * w.dstate / t_total, nthreads, desc
+
+
+def run_reference(args, world, rank):
+    """Reference arm: the fp64 oracle on the host cores, bounded samples."""
+    if rank != 0:
+        return
+    from selective_state_space_50_b200.workloads import WORKLOADS, generate
+    w = WORKLOADS[WORKLOAD]
+    inp = generate(w, channels=slice(0, 64))
+    wsub = w.replace(dim=64)
+    import oracle
+    nth = oracle.max_threads()
+    per_step = slice(0, 8)   # one step = 8 channels x all batch rows x full sequence
+    f64 = {k: v for k, v in inp.items() if k.endswith("_f64")}
+
+    def step():
+        sub = {}
+        for k, v in f64.items():
+            base = k[:-4]
+            if base in ("u", "delta", "z"):
+                sub[k] = np.ascontiguousarray(v[:, per_step])
+            elif base in ("A", "D", "delta_bias"):
+                sub[k] = np.ascontiguousarray(v[per_step])
+            else:
+                sub[k] = v
+        oracle.fwd(sub["u_f64"], sub["delta_f64"], sub["A_f64"], sub["B_f64"], sub["C_f64"],
+                   sub["D_f64"], sub["z_f64"], sub["delta_bias_f64"], True, nthreads=nth)
+    for _ in range(args.warmup):
+        step()
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t
+    elems = args.steps * w.batch * 8 * w.seqlen * w.dstate
+    v = elems / dt
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "dim": w.dim,
+                       "dstate": w.dstate, "io_dtype": w.io_dtype,
+                       "sample": "8 channels x 8 batch rows x 2048 steps per step"},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": nth, "kind": "oracle",
+                             "sample": f"{args.steps} steps of 8 channels x batch {w.batch} x "
+                                       f"seqlen {w.seqlen} of the {w.name} forward"},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, world, rank, local):
+    import torch
+    from selective_state_space_50_b200 import ssm_scan
+    from selective_state_space_50_b200.workloads import WORKLOADS, generate, to_torch
+
+    w = WORKLOADS[WORKLOAD]
+    dev = torch.device("cuda", local)
+    # every rank processes its own batch of the same shape (weak scaling)
+    w_rank = w.replace(seed=w.seed + 7919 * rank)
+    inp = generate(w_rank)
+    dv = to_torch(inp, w_rank, dev)
+    shape = ssm_scan.make_shape(w.batch, w.dim, w.seqlen, w.dstate, torch.bfloat16)
+    out = torch.empty_like(dv["u"])
+    last = torch.empty(w.batch, w.dim, w.dstate, device=dev, dtype=torch.float32)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def fwd():
+        ssm_scan.fwd_raw(shape, dv["u"], dv["delta"], dv["A"], dv["B"], dv["C"], dv["D"], dv["z"],
+                         dv["delta_bias"], True, out, last, None, stream)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        fwd()
+    torch.cuda.synchronize()
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    with ClockSampler(local) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record(stream)
+            fwd()
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    t_dev = sum(ms) / 1e3
+    t_max = max_over_ranks(t_dev, world)
+    elems_all = world * args.steps * w.batch * w.dim * w.seqlen * w.dstate
+
+    # ---- end to end through the binding, host buffers, copies inside the step
+    e2e_steps = max(5, min(args.steps, 50))
+    host = {k: dv[k].cpu().pin_memory() for k in ("u", "delta", "z", "B", "C", "A", "D",
+                                                   "delta_bias")}
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_h.numel() * out_h.element_size()
+    e_s = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
+    e_e = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
+    dtmp = {k: torch.empty_like(v) for k, v in dv.items() if v is not None}
+
+    def e2e_step():
+        for k, t in host.items():
+            dtmp[k].copy_(t, non_blocking=True)
+        o, _, _ = ssm_scan.selective_scan_fwd(dtmp["u"], dtmp["delta"], dtmp["A"], dtmp["B"],
+                                              dtmp["C"], dtmp["D"], dtmp["z"], dtmp["delta_bias"],
+                                              True, return_last_state=True, out=out)
+        out_h.copy_(o, non_blocking=True)
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    for i in range(e2e_steps):
+        flush.zero_()
+        e_s[i].record(stream)
+        e2e_step()
+        e_e[i].record(stream)
+    torch.cuda.synchronize()
+    t_e2e = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(e_s, e_e)) / 1e3, world)
+    e2e_val = world * e2e_steps * w.batch * w.dim * w.seqlen * w.dstate / t_e2e
+
+    if rank != 0:
+        return
+    peaks, peak_src = measured_peaks()
+    mean_s = t_dev / args.steps
+    ex2 = w.batch * w.dim * w.seqlen * w.dstate
+    sm_max = float(peaks.get("sm_max_mhz") or 1965.0)
+    mufu_peak = SM_COUNT_B200 * MUFU_EX2_PER_CLK_PER_SM * sm_max * 1e6
+    achieved = ex2 / mean_s
+    alg_bytes = algorithmic_bytes(w, 2)
+    traffic = None
+    tp = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tp):
+        with open(tp) as f:
+            traffic = json.load(f).get("ssm_fwd_" + WORKLOAD)
+    line = {
+        "metric": METRIC, "value": elems_all / t_max, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": max(3, args.warmup),
+        "ms_per_step": t_max / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "dim": w.dim,
+                   "dstate": w.dstate, "io_dtype": "bf16", "state_dtype": "f32",
+                   "parallelism": f"replicas x{world} (independent batches)",
+                   "l2": "flushed between steps (256 MiB write, outside the timed events)"},
+        "gbs": alg_bytes / mean_s / 1e9,
+        "roofline": {"bound": "alu", "achieved": achieved / 1e12, "peak": mufu_peak / 1e12,
+                     "unit": "Tex2/s", "frac": achieved / mufu_peak, "traffic": traffic,
+                     "peak_source": f"148 SMs x 16 ex2/clk x {sm_max:.0f} MHz (SFU)",
+                     "hbm": {"achieved_gbs": alg_bytes / mean_s / 1e9,
+                             "peak_gbs": float(peaks["hbm_gbs"]),
+                             "frac": alg_bytes / mean_s / 1e9 / float(peaks["hbm_gbs"]),
+                             "peak_source": peak_src, "alg_bytes": alg_bytes}},
+        "clocks": clk.summary(),
+        "e2e": {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        rate, cores, desc = cpu_oracle_rate(w, inp, args.cpu_budget)
+        line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                "sample": desc}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    args = ap.parse_args()
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

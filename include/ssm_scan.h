@@ -1,0 +1,159 @@
+/*
+ * ssm_scan.h -- C ABI of libssmscan.so, a selective-scan (S6) library for
+ * NVIDIA B200 (sm_100a).
+ *
+ * What the library computes (forward), per batch row b and channel d, for
+ * t = 0 .. seqlen-1, with n = 0 .. dstate-1:
+ *
+ *   Δ_t     = softplus(delta[b,d,t] + delta_bias[d])   (no softplus if the
+ *             flag is 0; bias treated as 0 if NULL)
+ *   Ā_t[n]  = exp(Δ_t A[d,n])
+ *   h_t[n]  = Ā_t[n] h_{t-1}[n] + Δ_t B[b,n,t] u[b,d,t],   h_{-1} = 0
+ *   y_t     = Σ_n C[b,n,t] h_t[n] + D[d] u[b,d,t]          (D term if D given)
+ *   out_t   = y_t · z_t · sigmoid(z_t)                      (if z given)
+ *
+ * Sources: booiljung.github.io, "3.2 선택적 스캔(Selective Scan) 알고리즘과
+ * 정보의 압축 및 선별" -- §1.1 (the recurrence and readout), §1.2 (selection:
+ * Δ_t = Softplus(Parameter + Linear_1(x_t)), B_t and C_t per token), §2.1
+ * (Ā_t = exp(Δ_t A) with diagonal A), §3.2 (fused kernel: only y reaches
+ * HBM), §3.3 (backward recomputes the states); 정보관리기술사 학습 노트,
+ * "상태공간 모델(SSM)과 Mamba 아키텍처", §3 (SiLU gate branch multiplied into
+ * the SSM output).  The input matrix is discretised as B̄_t = Δ_t B_t and the
+ * D skip term is added before the gate.
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    never allocates or frees device memory.  Layouts are dense row-major:
+ *      u, delta, z, out, dout       [batch][dim][seqlen]   io dtype
+ *      B, C                         [batch][dstate][seqlen] io dtype
+ *      A                            [dim][dstate]          float32
+ *      D, delta_bias                [dim]                  float32
+ *      last_state                   [batch][dim][dstate]   float32
+ *      ckpt                         [batch][dim][nchunk][dstate] float32,
+ *                                   nchunk = ceil(seqlen / SSM_CKPT_CHUNK)
+ *      du, ddelta, dz               [batch][dim][seqlen]   float32
+ *      dB, dC                       [batch][dstate][seqlen] float32
+ *      dA                           [dim][dstate]          float32
+ *      dD, ddelta_bias              [dim]                  float32
+ *    Pointers must be aligned to their element size.  The fast path (16-byte
+ *    vector loads and stores) is taken when every io tensor is 16-byte
+ *    aligned and seqlen * element size is a multiple of 16; otherwise the
+ *    same kernels use element-wise accesses.
+ *  - Pointers are checked with cudaPointerGetAttributes: host memory, or
+ *    memory of a device other than the current one, is refused with
+ *    SSM_ERR_INVALID_ARG before anything is launched.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
+ *    NULL is the legacy default stream).  The return value reports argument
+ *    and launch errors only; use the stream's own synchronisation to wait.
+ *  - On any error nothing is launched, and ssm_last_error_string() (per
+ *    calling thread) describes it.
+ *  - Supported: dstate in {1, 2, 4, 8, 16, 32}; io dtype float32 or bfloat16;
+ *    1 <= seqlen, batch, dim; batch * dim * seqlen < 2^31.
+ */
+#ifndef SSM_SCAN_H
+#define SSM_SCAN_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SSM_OK = 0,
+    SSM_ERR_INVALID_ARG = 1, /* null required pointer, bad size, misalignment */
+    SSM_ERR_UNSUPPORTED = 2, /* valid but not implemented (e.g. dstate = 3) */
+    SSM_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed */
+    SSM_ERR_TIMEOUT = 4      /* a bounded device-side wait gave up */
+} ssm_status_t;
+
+typedef enum { SSM_F32 = 0, SSM_BF16 = 1 } ssm_dtype_t;
+
+typedef struct {
+    int batch;            /* number of independent sequences */
+    int dim;              /* channels D (each has its own A row, D, bias) */
+    int seqlen;           /* L, time steps */
+    int dstate;           /* N, state size per channel */
+    ssm_dtype_t io_dtype; /* dtype of u, delta, z, B, C, out, dout */
+} ssm_shape_t;
+
+/* Steps between two saved states in the forward's checkpoint buffer. */
+#define SSM_CKPT_CHUNK 64
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int ssm_version(void);
+
+/* Message for the last error returned on this thread ("" if none). */
+const char *ssm_last_error_string(void);
+
+/*
+ * Bytes of the optional checkpoint buffer `ckpt` of ssm_selective_scan_fwd:
+ * batch * dim * ceil(seqlen / SSM_CKPT_CHUNK) * dstate * 4.
+ */
+ssm_status_t ssm_selective_scan_ckpt_bytes(const ssm_shape_t *shape, size_t *bytes);
+
+/*
+ * Forward selective scan (see the header comment for the arithmetic).
+ *
+ *  u, delta, A, B, C : required inputs.
+ *  D, z, delta_bias  : optional (NULL = term absent).
+ *  delta_softplus    : nonzero applies softplus to delta + delta_bias.
+ *  out               : required output, io dtype (may not alias an input).
+ *  last_state        : optional output, h_{seqlen-1}.
+ *  ckpt              : optional output; ckpt[b][d][k][:] = h at the last step
+ *                      of chunk k (step min(seqlen, (k+1)*SSM_CKPT_CHUNK) - 1).
+ *                      Pass it to ssm_selective_scan_bwd to skip the
+ *                      backward's state-recompute pre-pass.
+ * Errors: SSM_ERR_INVALID_ARG, SSM_ERR_UNSUPPORTED, SSM_ERR_CUDA.
+ */
+ssm_status_t ssm_selective_scan_fwd(const ssm_shape_t *shape,
+                                    const void *u, const void *delta,
+                                    const float *A, const void *B, const void *C,
+                                    const float *D, const void *z,
+                                    const float *delta_bias, int delta_softplus,
+                                    void *out, float *last_state, float *ckpt,
+                                    void *stream);
+
+/*
+ * Bytes of device scratch that ssm_selective_scan_bwd needs: 0 when the
+ * caller passes the forward's checkpoints (have_ckpt != 0), otherwise the
+ * size of a checkpoint buffer, which the backward fills itself first.
+ */
+ssm_status_t ssm_selective_scan_bwd_scratch_bytes(const ssm_shape_t *shape,
+                                                  int have_ckpt, size_t *bytes);
+
+/*
+ * Backward selective scan: given dout = dLoss/dout, writes the gradients of
+ * Loss with respect to every input of the forward.  The states are recomputed
+ * from the checkpoints (booiljung.github.io "3.2 Selective Scan" §3.3);
+ * nothing of size batch*dim*seqlen*dstate is ever stored.
+ *
+ *  u .. delta_softplus : the forward's inputs, unchanged.
+ *  dout                : required, io dtype.
+ *  ckpt                : the forward's checkpoint buffer, or NULL.
+ *  du, ddelta, dA, dB, dC : required outputs (float32, overwritten).
+ *  dD, dz, ddelta_bias : required iff D, z, delta_bias (resp.) are non-NULL,
+ *                        and must be NULL otherwise.
+ *  scratch, scratch_bytes : device scratch of at least
+ *                        ssm_selective_scan_bwd_scratch_bytes(shape, ckpt != NULL)
+ *                        bytes (may be NULL when that is 0).
+ * The gradient outputs must not alias each other or any input.
+ * Errors: SSM_ERR_INVALID_ARG, SSM_ERR_UNSUPPORTED, SSM_ERR_CUDA.
+ */
+ssm_status_t ssm_selective_scan_bwd(const ssm_shape_t *shape,
+                                    const void *u, const void *delta,
+                                    const float *A, const void *B, const void *C,
+                                    const float *D, const void *z,
+                                    const float *delta_bias, int delta_softplus,
+                                    const void *dout, const float *ckpt,
+                                    float *du, float *ddelta, float *dA,
+                                    float *dB, float *dC, float *dD, float *dz,
+                                    float *ddelta_bias,
+                                    void *scratch, size_t scratch_bytes,
+                                    void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSM_SCAN_H */

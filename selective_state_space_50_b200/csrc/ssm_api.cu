@@ -1,0 +1,231 @@
+// C ABI of libssmscan.so: argument checking and dispatch to the kernels.
+// Every check happens on the host before anything is launched, so a bad call
+// returns an error code instead of reaching the GPU.
+
+#include <stdarg.h>
+#include <stdint.h>
+#include <stdio.h>
+
+#include <string>
+
+#include "ssm_internal.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+ssm_status_t fail(ssm_status_t st, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
+ssm_status_t fail(ssm_status_t st, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return st;
+}
+
+ssm_status_t ok() {
+    g_last_error.clear();
+    return SSM_OK;
+}
+
+ssm_status_t cuda_fail(cudaError_t e, const char *what) {
+    return fail(SSM_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool supported_dstate(int n) {
+    return n == 1 || n == 2 || n == 4 || n == 8 || n == 16 || n == 32;
+}
+
+ssm_status_t check_shape(const ssm_shape_t *s) {
+    if (!s) return fail(SSM_ERR_INVALID_ARG, "shape is NULL");
+    if (s->batch < 1 || s->dim < 1 || s->seqlen < 1 || s->dstate < 1)
+        return fail(SSM_ERR_INVALID_ARG, "batch, dim, seqlen, dstate must be >= 1 (got %d, %d, %d, %d)",
+                    s->batch, s->dim, s->seqlen, s->dstate);
+    if (s->io_dtype != SSM_F32 && s->io_dtype != SSM_BF16)
+        return fail(SSM_ERR_INVALID_ARG, "io_dtype %d is not SSM_F32 or SSM_BF16", (int)s->io_dtype);
+    if ((long long)s->batch * s->dim * s->seqlen >= (1LL << 31))
+        return fail(SSM_ERR_UNSUPPORTED, "batch*dim*seqlen must be < 2^31");
+    if ((long long)s->batch * s->dstate * s->seqlen >= (1LL << 31))
+        return fail(SSM_ERR_UNSUPPORTED, "batch*dstate*seqlen must be < 2^31");
+    if (!supported_dstate(s->dstate))
+        return fail(SSM_ERR_UNSUPPORTED, "dstate %d not supported (1, 2, 4, 8, 16, 32)", s->dstate);
+    return SSM_OK;
+}
+
+// A pointer must be device (or managed) memory on the current device, aligned
+// to `align` bytes.  Host pointers are refused: handing one to a kernel would
+// fault the GPU.
+ssm_status_t check_ptr(const void *p, const char *name, size_t align, bool required) {
+    if (!p) {
+        if (required) return fail(SSM_ERR_INVALID_ARG, "%s is NULL", name);
+        return SSM_OK;
+    }
+    if ((uintptr_t)p % align)
+        return fail(SSM_ERR_INVALID_ARG, "%s is not %zu-byte aligned", name, align);
+    cudaPointerAttributes attr;
+    cudaError_t e = cudaPointerGetAttributes(&attr, p);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(SSM_ERR_INVALID_ARG, "%s: not a CUDA pointer (%s)", name, cudaGetErrorName(e));
+    }
+    if (attr.type != cudaMemoryTypeDevice && attr.type != cudaMemoryTypeManaged)
+        return fail(SSM_ERR_INVALID_ARG, "%s is not device memory", name);
+    int dev = -1;
+    cudaGetDevice(&dev);
+    if (attr.type == cudaMemoryTypeDevice && attr.device != dev)
+        return fail(SSM_ERR_INVALID_ARG, "%s lives on device %d, current device is %d", name,
+                    attr.device, dev);
+    return SSM_OK;
+}
+
+#define SSM_TRY(expr)                    \
+    do {                                 \
+        ssm_status_t st_ = (expr);       \
+        if (st_ != SSM_OK) return st_;   \
+    } while (0)
+
+size_t esize(ssm_dtype_t t) { return t == SSM_BF16 ? 2 : 4; }
+
+int n_ckpt(const ssm_shape_t *s) { return (s->seqlen + SSM_CKPT_CHUNK - 1) / SSM_CKPT_CHUNK; }
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+int ssm_version(void) { return 100; }
+
+const char *ssm_last_error_string(void) { return g_last_error.c_str(); }
+
+ssm_status_t ssm_selective_scan_ckpt_bytes(const ssm_shape_t *shape, size_t *bytes) {
+    SSM_TRY(check_shape(shape));
+    if (!bytes) return fail(SSM_ERR_INVALID_ARG, "bytes is NULL");
+    *bytes = (size_t)shape->batch * shape->dim * n_ckpt(shape) * shape->dstate * sizeof(float);
+    return ok();
+}
+
+ssm_status_t ssm_selective_scan_bwd_scratch_bytes(const ssm_shape_t *shape, int have_ckpt,
+                                                  size_t *bytes) {
+    SSM_TRY(check_shape(shape));
+    if (!bytes) return fail(SSM_ERR_INVALID_ARG, "bytes is NULL");
+    *bytes = have_ckpt ? 0
+                       : (size_t)shape->batch * shape->dim * n_ckpt(shape) * shape->dstate * sizeof(float);
+    return ok();
+}
+
+ssm_status_t ssm_selective_scan_fwd(const ssm_shape_t *shape, const void *u, const void *delta,
+                                    const float *A, const void *B, const void *C, const float *D,
+                                    const void *z, const float *delta_bias, int delta_softplus,
+                                    void *out, float *last_state, float *ckpt, void *stream) {
+    SSM_TRY(check_shape(shape));
+    const size_t es = esize(shape->io_dtype);
+    SSM_TRY(check_ptr(u, "u", es, true));
+    SSM_TRY(check_ptr(delta, "delta", es, true));
+    SSM_TRY(check_ptr(A, "A", 4, true));
+    SSM_TRY(check_ptr(B, "B", es, true));
+    SSM_TRY(check_ptr(C, "C", es, true));
+    SSM_TRY(check_ptr(D, "D", 4, false));
+    SSM_TRY(check_ptr(z, "z", es, false));
+    SSM_TRY(check_ptr(delta_bias, "delta_bias", 4, false));
+    SSM_TRY(check_ptr(out, "out", es, true));
+    SSM_TRY(check_ptr(last_state, "last_state", 4, false));
+    SSM_TRY(check_ptr(ckpt, "ckpt", 4, false));
+    if (out == u || out == delta || out == z || out == B || out == C)
+        return fail(SSM_ERR_INVALID_ARG, "out may not alias an input");
+
+    ssm::FwdParams p{};
+    p.u = u; p.delta = delta; p.A = A; p.B = B; p.C = C; p.D = D; p.z = z;
+    p.delta_bias = delta_bias; p.out = out; p.last_state = last_state; p.ckpt = ckpt;
+    p.batch = shape->batch; p.dim = shape->dim; p.L = shape->seqlen; p.N = shape->dstate;
+    p.n_ckpt = n_ckpt(shape);
+    p.softplus = delta_softplus != 0;
+    p.io_bf16 = shape->io_dtype == SSM_BF16;
+    p.vec_ok = ((size_t)shape->seqlen * es) % 16 == 0 && aligned16(u) && aligned16(delta) &&
+               aligned16(B) && aligned16(C) && aligned16(out) && (!z || aligned16(z));
+    cudaError_t e = ssm::launch_fwd(p, false, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "ssm_selective_scan_fwd launch");
+    return ok();
+}
+
+ssm_status_t ssm_selective_scan_bwd(const ssm_shape_t *shape, const void *u, const void *delta,
+                                    const float *A, const void *B, const void *C, const float *D,
+                                    const void *z, const float *delta_bias, int delta_softplus,
+                                    const void *dout, const float *ckpt, float *du, float *ddelta,
+                                    float *dA, float *dB, float *dC, float *dD, float *dz,
+                                    float *ddelta_bias, void *scratch, size_t scratch_bytes,
+                                    void *stream) {
+    SSM_TRY(check_shape(shape));
+    const size_t es = esize(shape->io_dtype);
+    SSM_TRY(check_ptr(u, "u", es, true));
+    SSM_TRY(check_ptr(delta, "delta", es, true));
+    SSM_TRY(check_ptr(A, "A", 4, true));
+    SSM_TRY(check_ptr(B, "B", es, true));
+    SSM_TRY(check_ptr(C, "C", es, true));
+    SSM_TRY(check_ptr(D, "D", 4, false));
+    SSM_TRY(check_ptr(z, "z", es, false));
+    SSM_TRY(check_ptr(delta_bias, "delta_bias", 4, false));
+    SSM_TRY(check_ptr(dout, "dout", es, true));
+    SSM_TRY(check_ptr(ckpt, "ckpt", 4, false));
+    SSM_TRY(check_ptr(du, "du", 4, true));
+    SSM_TRY(check_ptr(ddelta, "ddelta", 4, true));
+    SSM_TRY(check_ptr(dA, "dA", 4, true));
+    SSM_TRY(check_ptr(dB, "dB", 4, true));
+    SSM_TRY(check_ptr(dC, "dC", 4, true));
+    SSM_TRY(check_ptr(dD, "dD", 4, D != nullptr));
+    SSM_TRY(check_ptr(dz, "dz", 4, z != nullptr));
+    SSM_TRY(check_ptr(ddelta_bias, "ddelta_bias", 4, delta_bias != nullptr));
+    if (!D && dD) return fail(SSM_ERR_INVALID_ARG, "dD given without D");
+    if (!z && dz) return fail(SSM_ERR_INVALID_ARG, "dz given without z");
+    if (!delta_bias && ddelta_bias)
+        return fail(SSM_ERR_INVALID_ARG, "ddelta_bias given without delta_bias");
+
+    const int nck = n_ckpt(shape);
+    const size_t ck_bytes = (size_t)shape->batch * shape->dim * nck * shape->dstate * sizeof(float);
+    float *ck = const_cast<float *>(ckpt);
+    if (!ckpt) {
+        if (scratch_bytes < ck_bytes)
+            return fail(SSM_ERR_INVALID_ARG, "scratch_bytes %zu < required %zu (no ckpt given)",
+                        scratch_bytes, ck_bytes);
+        SSM_TRY(check_ptr(scratch, "scratch", 16, true));
+        ck = static_cast<float *>(scratch);
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const bool vec_ok = ((size_t)shape->seqlen * es) % 16 == 0 && aligned16(u) && aligned16(delta) &&
+                        aligned16(B) && aligned16(C) && aligned16(dout) && (!z || aligned16(z));
+    if (!ckpt) {
+        ssm::FwdParams fp{};
+        fp.u = u; fp.delta = delta; fp.A = A; fp.B = B; fp.C = C; fp.D = D; fp.z = z;
+        fp.delta_bias = delta_bias; fp.out = nullptr; fp.last_state = nullptr; fp.ckpt = ck;
+        fp.batch = shape->batch; fp.dim = shape->dim; fp.L = shape->seqlen; fp.N = shape->dstate;
+        fp.n_ckpt = nck; fp.softplus = delta_softplus != 0;
+        fp.io_bf16 = shape->io_dtype == SSM_BF16; fp.vec_ok = vec_ok;
+        cudaError_t e = ssm::launch_fwd(fp, true, st);
+        if (e != cudaSuccess) return cuda_fail(e, "ssm_selective_scan_bwd state pass");
+    }
+    // gradients accumulated with atomics start from zero
+    const size_t bcl = (size_t)shape->batch * shape->dstate * shape->seqlen * sizeof(float);
+    cudaError_t e = cudaSuccess;
+    if (e == cudaSuccess) e = cudaMemsetAsync(dA, 0, (size_t)shape->dim * shape->dstate * 4, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dB, 0, bcl, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dC, 0, bcl, st);
+    if (e == cudaSuccess && dD) e = cudaMemsetAsync(dD, 0, (size_t)shape->dim * 4, st);
+    if (e == cudaSuccess && ddelta_bias) e = cudaMemsetAsync(ddelta_bias, 0, (size_t)shape->dim * 4, st);
+    if (e != cudaSuccess) return cuda_fail(e, "ssm_selective_scan_bwd memset");
+
+    ssm::BwdParams p{};
+    p.u = u; p.delta = delta; p.A = A; p.B = B; p.C = C; p.D = D; p.z = z;
+    p.delta_bias = delta_bias; p.dout = dout; p.ckpt = ck;
+    p.du = du; p.ddelta = ddelta; p.dA = dA; p.dB = dB; p.dC = dC; p.dD = dD; p.dz = dz;
+    p.ddelta_bias = ddelta_bias;
+    p.batch = shape->batch; p.dim = shape->dim; p.L = shape->seqlen; p.N = shape->dstate;
+    p.n_ckpt = nck; p.softplus = delta_softplus != 0;
+    p.io_bf16 = shape->io_dtype == SSM_BF16; p.vec_ok = vec_ok;
+    e = ssm::launch_bwd(p, st);
+    if (e != cudaSuccess) return cuda_fail(e, "ssm_selective_scan_bwd launch");
+    return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,110 @@
+// Device helpers shared by the selective-scan kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#define SSM_LOG2E 1.4426950408889634f
+
+namespace ssm {
+
+// 2^x on the MUFU (SFU) pipe: the PTX instruction ex2.approx.ftz.f32.
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// softplus(r) = log(1 + e^r).  Above r = 20, log1p(e^r) - r = log1p(e^-r) is
+// below 2.1e-9, under half an ulp of r in fp32, so r itself is returned.
+__device__ __forceinline__ float softplus(float r) {
+    return r > 20.f ? r : log1pf(__expf(r));
+}
+
+__device__ __forceinline__ float sigmoid(float v) {
+    return __fdividef(1.f, 1.f + __expf(-v));
+}
+
+// ---- io element types -------------------------------------------------------
+
+template <typename T> struct IO;
+
+template <> struct IO<float> {
+    static constexpr int kVec = 4;  // elements per 16-byte vector
+    __device__ __forceinline__ static float to_f(float v) { return v; }
+    __device__ __forceinline__ static float from_f(float v) { return v; }
+    // 16-byte vector <-> 4 floats
+    __device__ __forceinline__ static void unpack(const uint4 &q, float *f) {
+        f[0] = __uint_as_float(q.x); f[1] = __uint_as_float(q.y);
+        f[2] = __uint_as_float(q.z); f[3] = __uint_as_float(q.w);
+    }
+    __device__ __forceinline__ static uint4 pack(const float *f) {
+        return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]),
+                          __float_as_uint(f[2]), __float_as_uint(f[3]));
+    }
+};
+
+template <> struct IO<__nv_bfloat16> {
+    static constexpr int kVec = 8;
+    __device__ __forceinline__ static float to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
+    __device__ __forceinline__ static __nv_bfloat16 from_f(float v) { return __float2bfloat16_rn(v); }
+    __device__ __forceinline__ static void unpack(const uint4 &q, float *f) {
+        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            f[2 * i] = __uint_as_float(w[i] << 16);
+            f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
+    }
+    __device__ __forceinline__ static uint32_t pack2(float lo, float hi) {
+        __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+        return *reinterpret_cast<uint32_t *>(&v);
+    }
+    __device__ __forceinline__ static uint4 pack(const float *f) {
+        return make_uint4(pack2(f[0], f[1]), pack2(f[2], f[3]), pack2(f[4], f[5]),
+                          pack2(f[6], f[7]));
+    }
+};
+
+// Loads kVec consecutive elements starting at p[0] into f (as fp32).  Elements
+// at index >= n (n < kVec at a ragged end) read as `fill`.  `vec` says the
+// 16-byte load is legal (aligned and fully in range).
+template <typename T>
+__device__ __forceinline__ void load_vec(const T *p, int n, bool vec, float fill, float *f) {
+    constexpr int V = IO<T>::kVec;
+    if (vec && n >= V) {
+        uint4 q = __ldg(reinterpret_cast<const uint4 *>(p));
+        IO<T>::unpack(q, f);
+    } else {
+#pragma unroll
+        for (int i = 0; i < V; ++i) f[i] = i < n ? IO<T>::to_f(p[i]) : fill;
+    }
+}
+
+// Streaming variant (evict-first): for data read exactly once.
+template <typename T>
+__device__ __forceinline__ void load_vec_stream(const T *p, int n, bool vec, float fill, float *f) {
+    constexpr int V = IO<T>::kVec;
+    if (vec && n >= V) {
+        uint4 q = __ldcs(reinterpret_cast<const uint4 *>(p));
+        IO<T>::unpack(q, f);
+    } else {
+#pragma unroll
+        for (int i = 0; i < V; ++i) f[i] = i < n ? IO<T>::to_f(p[i]) : fill;
+    }
+}
+
+template <typename T>
+__device__ __forceinline__ void store_vec(T *p, int n, bool vec, const float *f) {
+    constexpr int V = IO<T>::kVec;
+    if (vec && n >= V) {
+        __stcs(reinterpret_cast<uint4 *>(p), IO<T>::pack(f));
+    } else {
+#pragma unroll
+        for (int i = 0; i < V; ++i)
+            if (i < n) p[i] = IO<T>::from_f(f[i]);
+    }
+}
+
+}  // namespace ssm

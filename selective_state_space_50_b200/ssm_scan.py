@@ -1,0 +1,186 @@
+"""Python binding of libssmscan.so (the C ABI in include/ssm_scan.h).
+
+Argument marshalling only: torch provides device memory and the current CUDA
+stream; every step of the scan runs in the library's kernels.  There is no
+fallback implementation: if the shared library is missing or cannot be
+loaded, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libssmscan.so")
+
+SSM_OK, SSM_ERR_INVALID_ARG, SSM_ERR_UNSUPPORTED, SSM_ERR_CUDA, SSM_ERR_TIMEOUT = range(5)
+SSM_F32, SSM_BF16 = 0, 1
+CKPT_CHUNK = 64  # SSM_CKPT_CHUNK in include/ssm_scan.h
+
+EXPORTS = ("ssm_version", "ssm_last_error_string", "ssm_selective_scan_ckpt_bytes",
+           "ssm_selective_scan_fwd", "ssm_selective_scan_bwd_scratch_bytes",
+           "ssm_selective_scan_bwd")
+
+
+class SSMError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"ssm status {status}: {msg}")
+        self.status = status
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int), ("dim", ctypes.c_int), ("seqlen", ctypes.c_int),
+                ("dstate", ctypes.c_int), ("io_dtype", ctypes.c_int)]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Loads the library (once) and declares the C signatures."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with "
+                           "`python -m selective_state_space_50_b200.build`")
+    lib = ctypes.CDLL(path)
+    vp, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    sp = ctypes.POINTER(Shape)
+    lib.ssm_version.restype = i
+    lib.ssm_last_error_string.restype = ctypes.c_char_p
+    lib.ssm_selective_scan_ckpt_bytes.argtypes = [sp, ctypes.POINTER(sz)]
+    lib.ssm_selective_scan_ckpt_bytes.restype = i
+    lib.ssm_selective_scan_bwd_scratch_bytes.argtypes = [sp, i, ctypes.POINTER(sz)]
+    lib.ssm_selective_scan_bwd_scratch_bytes.restype = i
+    lib.ssm_selective_scan_fwd.argtypes = [sp] + [vp] * 8 + [i] + [vp] * 4
+    lib.ssm_selective_scan_fwd.restype = i
+    lib.ssm_selective_scan_bwd.argtypes = [sp] + [vp] * 8 + [i] + [vp] * 11 + [sz, vp]
+    lib.ssm_selective_scan_bwd.restype = i
+    _lib = lib
+    return lib
+
+
+def last_error() -> str:
+    return load_library().ssm_last_error_string().decode()
+
+
+def _check(status: int):
+    if status != SSM_OK:
+        raise SSMError(status, last_error())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_ptr(stream: Optional[torch.cuda.Stream]):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def make_shape(batch, dim, seqlen, dstate, io_dtype) -> Shape:
+    if isinstance(io_dtype, torch.dtype):
+        io_dtype = {torch.float32: SSM_F32, torch.bfloat16: SSM_BF16}[io_dtype]
+    return Shape(batch, dim, seqlen, dstate, io_dtype)
+
+
+def ckpt_numel(shape: Shape) -> int:
+    n = ctypes.c_size_t()
+    _check(load_library().ssm_selective_scan_ckpt_bytes(ctypes.byref(shape), ctypes.byref(n)))
+    return n.value // 4
+
+
+def bwd_scratch_bytes(shape: Shape, have_ckpt: bool) -> int:
+    n = ctypes.c_size_t()
+    _check(load_library().ssm_selective_scan_bwd_scratch_bytes(ctypes.byref(shape),
+                                                               int(bool(have_ckpt)),
+                                                               ctypes.byref(n)))
+    return n.value
+
+
+def _shape_of(u: torch.Tensor, A: torch.Tensor) -> Shape:
+    if u.dim() != 3 or A.dim() != 2:
+        raise ValueError("u must be [batch, dim, seqlen] and A [dim, dstate]")
+    return make_shape(u.shape[0], u.shape[1], u.shape[2], A.shape[1], u.dtype)
+
+
+def fwd_raw(shape: Shape, u, delta, A, B, C, D, z, delta_bias, delta_softplus: bool,
+            out, last_state, ckpt, stream=None):
+    """Direct C-ABI call on raw tensors (no checks beyond the library's own)."""
+    _check(load_library().ssm_selective_scan_fwd(
+        ctypes.byref(shape), _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+        _ptr(delta_bias), int(bool(delta_softplus)), _ptr(out), _ptr(last_state), _ptr(ckpt),
+        _stream_ptr(stream)))
+
+
+def bwd_raw(shape: Shape, u, delta, A, B, C, D, z, delta_bias, delta_softplus: bool, dout,
+            ckpt, du, ddelta, dA, dB, dC, dD, dz, ddelta_bias, scratch, stream=None):
+    nbytes = 0 if scratch is None else scratch.numel() * scratch.element_size()
+    _check(load_library().ssm_selective_scan_bwd(
+        ctypes.byref(shape), _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+        _ptr(delta_bias), int(bool(delta_softplus)), _ptr(dout), _ptr(ckpt), _ptr(du),
+        _ptr(ddelta), _ptr(dA), _ptr(dB), _ptr(dC), _ptr(dD), _ptr(dz), _ptr(ddelta_bias),
+        _ptr(scratch), ctypes.c_size_t(nbytes), _stream_ptr(stream)))
+
+
+def _need(t, name, dtype=None, cuda=True):
+    if t is None:
+        return
+    if cuda and not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None,
+                       delta_softplus: bool = True, return_last_state: bool = False,
+                       return_ckpt: bool = False, out=None, stream=None):
+    """Forward selective scan.  u, delta, z, B, C share one io dtype (float32 or
+    bfloat16); A, D, delta_bias are float32.  Returns (out, last_state, ckpt)
+    with the last two None unless requested."""
+    io = u.dtype
+    for t, n in ((u, "u"), (delta, "delta"), (B, "B"), (C, "C"), (z, "z")):
+        _need(t, n, io)
+    for t, n in ((A, "A"), (D, "D"), (delta_bias, "delta_bias")):
+        _need(t, n, torch.float32)
+    shape = _shape_of(u, A)
+    if out is None:
+        out = torch.empty_like(u)
+    last = (torch.empty(shape.batch, shape.dim, shape.dstate, device=u.device,
+                        dtype=torch.float32) if return_last_state else None)
+    ck = (torch.empty(ckpt_numel(shape), device=u.device, dtype=torch.float32)
+          if return_ckpt else None)
+    fwd_raw(shape, u, delta, A, B, C, D, z, delta_bias, delta_softplus, out, last, ck, stream)
+    return out, last, ck
+
+
+def selective_scan_bwd(u, delta, A, B, C, D, z, delta_bias, delta_softplus: bool, dout,
+                       ckpt=None, stream=None):
+    """Backward selective scan; returns a dict of float32 gradients (du, ddelta,
+    dA, dB, dC and, for the optional inputs that were given, dD, dz,
+    ddelta_bias)."""
+    io = u.dtype
+    for t, n in ((u, "u"), (delta, "delta"), (B, "B"), (C, "C"), (z, "z"), (dout, "dout")):
+        _need(t, n, io)
+    for t, n in ((A, "A"), (D, "D"), (delta_bias, "delta_bias"), (ckpt, "ckpt")):
+        _need(t, n, torch.float32)
+    shape = _shape_of(u, A)
+    f32 = dict(device=u.device, dtype=torch.float32)
+    g = {"du": torch.empty(u.shape, **f32), "ddelta": torch.empty(u.shape, **f32),
+         "dA": torch.empty(A.shape, **f32), "dB": torch.empty(B.shape, **f32),
+         "dC": torch.empty(C.shape, **f32),
+         "dD": torch.empty(D.shape, **f32) if D is not None else None,
+         "dz": torch.empty(u.shape, **f32) if z is not None else None,
+         "ddelta_bias": torch.empty(delta_bias.shape, **f32) if delta_bias is not None else None}
+    nscratch = bwd_scratch_bytes(shape, ckpt is not None)
+    scratch = torch.empty(max(1, nscratch // 4), **f32) if nscratch else None
+    bwd_raw(shape, u, delta, A, B, C, D, z, delta_bias, delta_softplus, dout, ckpt,
+            g["du"], g["ddelta"], g["dA"], g["dB"], g["dC"], g["dD"], g["dz"],
+            g["ddelta_bias"], scratch, stream)
+    return {k: v for k, v in g.items() if v is not None}

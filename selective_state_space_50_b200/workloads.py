@@ -23,8 +23,10 @@ Tensor layouts (all row-major / C-contiguous):
 """
 from __future__ import annotations
 
+import concurrent.futures as _cf
 import dataclasses
 import math
+import os
 from typing import Dict, Optional
 
 import numpy as np
@@ -60,12 +62,25 @@ def _uniform_block(key: np.uint64, start: int, count: int) -> np.ndarray:
     return (x >> np.uint64(11)).astype(np.float64) * (1.0 / 9007199254740992.0)
 
 
+def _parallel(fn, starts):
+    """Runs fn(start) for every chunk start; numpy releases the GIL inside the
+    ufuncs, so chunks run concurrently.  Results do not depend on scheduling."""
+    if len(starts) <= 1:
+        for s in starts:
+            fn(s)
+        return
+    with _cf.ThreadPoolExecutor(max_workers=min(len(starts), os.cpu_count() or 1)) as ex:
+        list(ex.map(fn, starts))
+
+
 def uniform(seed: int, stream: int, n: int, lo: float = 0.0, hi: float = 1.0) -> np.ndarray:
     key = _key(seed, stream)
     out = np.empty(n, dtype=np.float64)
-    for s in range(0, n, _CHUNK):
+
+    def fill(s):
         c = min(_CHUNK, n - s)
         out[s:s + c] = lo + (hi - lo) * _uniform_block(key, s, c)
+    _parallel(fill, list(range(0, n, _CHUNK)))
     return out
 
 
@@ -74,7 +89,8 @@ def normal(seed: int, stream: int, n: int, std: float = 1.0) -> np.ndarray:
     key = _key(seed, stream)
     out = np.empty(n, dtype=np.float64)
     npairs = (n + 1) // 2
-    for s in range(0, npairs, _CHUNK):
+
+    def fill(s):
         c = min(_CHUNK, npairs - s)
         uu = _uniform_block(key, 2 * s, 2 * c).reshape(c, 2)
         r = np.sqrt(-2.0 * np.log1p(-uu[:, 0]))  # 1-u1 in (0, 1]
@@ -85,8 +101,9 @@ def normal(seed: int, stream: int, n: int, std: float = 1.0) -> np.ndarray:
         flat = pair.reshape(-1)
         lo = 2 * s
         take = min(2 * c, n - lo)
-        out[lo:lo + take] = flat[:take]
-    return out * std
+        out[lo:lo + take] = flat[:take] * std
+    _parallel(fill, list(range(0, npairs, _CHUNK)))
+    return out
 
 
 # ---------------------------------------------------------------- bf16 rounding
@@ -127,6 +144,7 @@ class Workload:
     A_dist: str = "neg_n1"   # "neg_n1": A[d,n] = -(n+1); "neg_lognormal": -exp(N(0,1))
     bias_dist: str = "expm1_u"   # "expm1_u": log(expm1(U[1e-3, 0.1])); "long_memory"
     delta_std: float = 1.0
+    delta_abs: bool = False  # |N(0, std)| raw deltas (for callers passing Δ without softplus)
 
     @property
     def elems(self) -> int:
@@ -212,6 +230,8 @@ def generate(w: Workload, with_dout: bool = False,
     names = ["u", "delta", "z"] + (["dout"] if with_dout else [])
     for name in names:
         x = per_channel(STREAMS[name], w.delta_std if name == "delta" else 1.0)
+        if name == "delta" and w.delta_abs:
+            x = np.abs(x)
         dev, f64 = _cast(x, w.io_dtype)
         out[name], out[name + "_f64"] = dev, f64
     for name in ("B", "C"):
@@ -227,3 +247,23 @@ def generate(w: Workload, with_dout: bool = False,
             elif base in ("A", "D", "delta_bias"):
                 out[name] = np.ascontiguousarray(out[name][channels])
     return out
+
+
+def to_torch(inputs: Dict[str, np.ndarray], w: Workload, device):
+    """Device tensors (io dtype / fp32) of a generated workload; optional
+    inputs the workload leaves out map to None."""
+    import torch
+
+    def dev(x):
+        if x.dtype == np.uint16:
+            return torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(device)
+        return torch.from_numpy(np.ascontiguousarray(x)).to(device)
+    d = {k: dev(inputs[k]) for k in ("u", "delta", "z", "B", "C", "dout", "A", "D", "delta_bias")
+         if k in inputs}
+    if not w.has_z:
+        d["z"] = None
+    if not w.has_D:
+        d["D"] = None
+    if not w.has_bias:
+        d["delta_bias"] = None
+    return d

@@ -1,0 +1,187 @@
+"""GPU parity: the CUDA library (called through its C ABI) against the fp64
+oracle on the same seeded inputs.  Tolerances are documented in helpers.py."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from selective_state_space_50_b200 import ssm_scan
+from selective_state_space_50_b200.workloads import WORKLOADS, Workload, generate
+
+from helpers import (assert_close_grad, assert_close_io, subset_channels, to_device, to_f64)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    ssm_scan.load_library()
+
+
+def run_fwd(dv, w, **kw):
+    out, last, ck = ssm_scan.selective_scan_fwd(dv["u"], dv["delta"], dv["A"], dv["B"], dv["C"],
+                                                dv["D"], dv["z"], dv["delta_bias"], w.softplus,
+                                                return_last_state=True, **kw)
+    torch.cuda.synchronize()
+    return out, last, ck
+
+
+def check_fwd(w: Workload, channels=None):
+    inp = generate(w)
+    dv = to_device(inp, w)
+    out, last, _ = run_fwd(dv, w)
+    if channels is not None:
+        sub = subset_channels(inp, channels)
+        ref, rlast = oracle.fwd_workload(sub, w)
+        got = to_f64(out)[:, channels]
+        glast = to_f64(last)[:, channels]
+    else:
+        ref, rlast = oracle.fwd_workload(inp, w)
+        got, glast = to_f64(out), to_f64(last)
+    e = assert_close_io(got, ref, w.io_dtype)
+    # the final state is fp32 in any io dtype
+    assert_close_io(glast, rlast, "f32" if w.io_dtype == "f32" else "bf16", "last_state")
+    return e
+
+
+def test_fwd_tiny_f32():
+    check_fwd(WORKLOADS["tiny_f32"])
+
+
+@pytest.mark.parametrize("name", ["mamba130m_layer", "mamba2p8b_layer"])
+def test_fwd_layer_shapes_full(name):
+    check_fwd(WORKLOADS[name])
+
+
+def test_fwd_long_context_sampled_channels():
+    w = WORKLOADS["long_context"]
+    check_fwd(w, channels=slice(0, w.dim, 97))
+
+
+SMALL = [
+    # batch, dim, L, N, io, z, D, bias, softplus, A_dist
+    (1, 1, 1, 16, "f32", True, True, True, True, "neg_lognormal"),
+    (2, 5, 7, 16, "f32", True, True, True, True, "neg_lognormal"),
+    (1, 37, 33, 16, "bf16", True, True, True, True, "neg_lognormal"),
+    (3, 19, 100, 8, "f32", False, True, True, True, "neg_lognormal"),
+    (2, 9, 1023, 32, "f32", True, False, False, False, "neg_lognormal"),
+    (1, 130, 64, 4, "bf16", True, True, True, True, "neg_n1"),
+    (2, 7, 129, 2, "f32", True, True, True, True, "neg_lognormal"),
+    (2, 7, 129, 1, "bf16", False, False, True, True, "neg_lognormal"),
+    (1, 2048, 300, 16, "bf16", True, True, True, True, "neg_lognormal"),   # few (b,d): per-state lanes
+    (1, 1000, 77, 32, "f32", True, True, True, True, "neg_lognormal"),
+    (1, 1000, 77, 8, "f32", True, True, True, True, "neg_lognormal"),
+    (1, 1000, 77, 4, "f32", True, True, True, True, "neg_lognormal"),
+]
+
+
+def small_workload(batch, dim, L, N, io, z, D, bias, sp, A_dist, seed=77):
+    # without softplus the caller supplies the step size itself: draw it >= 0
+    # (a negative step makes Ā > 1 and the state grows without bound)
+    return Workload("small", batch, L, dim, N, io, seed=seed, has_z=z, has_D=D, has_bias=bias,
+                    softplus=sp, A_dist=A_dist, D_dist="u0.5_1.5",
+                    delta_abs=not sp, delta_std=1.0 if sp else 0.1)
+
+
+@pytest.mark.parametrize("case", SMALL)
+def test_fwd_small_and_ragged(case):
+    check_fwd(small_workload(*case))
+
+
+def test_fwd_ckpt_holds_chunk_end_states():
+    w = small_workload(2, 6, 200, 16, "f32", True, True, True, True, "neg_lognormal")
+    inp = generate(w)
+    dv = to_device(inp, w)
+    out, last, ck = run_fwd(dv, w, return_ckpt=True)
+    ck = to_f64(ck).reshape(2, 6, -1, 16)
+    assert ck.shape[2] == math.ceil(200 / ssm_scan.CKPT_CHUNK)
+    for k in range(ck.shape[2]):
+        tend = min(200, (k + 1) * ssm_scan.CKPT_CHUNK)
+        _, st = oracle.fwd(inp["u_f64"][..., :tend], inp["delta_f64"][..., :tend], inp["A_f64"],
+                           inp["B_f64"][..., :tend], inp["C_f64"][..., :tend], inp["D_f64"],
+                           inp["z_f64"][..., :tend], inp["delta_bias_f64"], True)
+        assert_close_io(ck[:, :, k], st, "f32", f"ckpt[{k}]")
+
+
+def test_fwd_unaligned_rows_use_elementwise_path():
+    """Rows that are not 16-byte aligned (odd L, offset base) still match."""
+    w = small_workload(2, 5, 61, 16, "bf16", True, True, True, True, "neg_lognormal")
+    inp = generate(w)
+    dv = to_device(inp, w)
+    shifted = {}
+    for k in ("u", "delta", "z", "B", "C"):
+        t = dv[k]
+        buf = torch.empty(t.numel() + 1, dtype=t.dtype, device=t.device)
+        v = buf[1:].view(t.shape)
+        v.copy_(t)
+        shifted[k] = v
+    dv.update(shifted)
+    out, last, _ = run_fwd(dv, w)
+    ref, rlast = oracle.fwd_workload(inp, w)
+    assert_close_io(to_f64(out), ref, "bf16")
+
+
+def test_fwd_on_side_stream():
+    w = small_workload(2, 33, 150, 16, "f32", True, True, True, True, "neg_lognormal")
+    inp = generate(w)
+    dv = to_device(inp, w)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        out, last, _ = ssm_scan.selective_scan_fwd(dv["u"], dv["delta"], dv["A"], dv["B"],
+                                                   dv["C"], dv["D"], dv["z"], dv["delta_bias"],
+                                                   True, return_last_state=True)
+    s.synchronize()
+    ref, _ = oracle.fwd_workload(inp, w)
+    assert_close_io(to_f64(out), ref, "f32")
+
+
+def test_fwd_repeatable_bitwise():
+    w = small_workload(2, 40, 300, 16, "bf16", True, True, True, True, "neg_lognormal")
+    dv = to_device(generate(w), w)
+    o1, _, _ = run_fwd(dv, w)
+    o2, _, _ = run_fwd(dv, w)
+    assert torch.equal(o1, o2)
+
+
+# ------------------------------------------------------------------ backward
+
+def check_bwd(w: Workload, use_ckpt: bool):
+    inp = generate(w, with_dout=True)
+    dv = to_device(inp, w)
+    ck = None
+    if use_ckpt:
+        _, _, ck = run_fwd(dv, w, return_ckpt=True)
+    g = ssm_scan.selective_scan_bwd(dv["u"], dv["delta"], dv["A"], dv["B"], dv["C"], dv["D"],
+                                    dv["z"], dv["delta_bias"], w.softplus, dv["dout"], ckpt=ck)
+    torch.cuda.synchronize()
+    ref = oracle.bwd_workload(inp, w)
+    assert set(g) == set(ref)
+    errs = {}
+    for k in ref:
+        errs[k] = assert_close_grad(to_f64(g[k]), ref[k], k)
+    return errs
+
+
+BWD_SMALL = [
+    (1, 3, 12, 4, "f32", True, True, True, True, "neg_lognormal"),
+    (2, 5, 70, 16, "f32", True, True, True, True, "neg_lognormal"),
+    (2, 37, 200, 16, "bf16", True, True, True, True, "neg_lognormal"),
+    (1, 9, 129, 8, "f32", False, False, False, False, "neg_lognormal"),
+    (2, 17, 64, 32, "f32", True, True, True, True, "neg_lognormal"),
+    (1, 70, 100, 2, "bf16", True, True, True, True, "neg_lognormal"),
+    (1, 70, 100, 1, "f32", True, False, True, True, "neg_lognormal"),
+]
+
+
+@pytest.mark.parametrize("case", BWD_SMALL)
+@pytest.mark.parametrize("use_ckpt", [True, False])
+def test_bwd_small(case, use_ckpt):
+    check_bwd(small_workload(*case), use_ckpt)
+
+
+def test_bwd_layer_shape_full():
+    check_bwd(WORKLOADS["mamba130m_layer_fwdbwd"], use_ckpt=True)
