@@ -152,6 +152,16 @@ ssm_status_t ssm_selective_scan_bwd(const ssm_shape_t *shape,
                                     void *scratch, size_t scratch_bytes,
                                     void *stream);
 
+/*
+ * Synchronises `stream`, then reports (and clears) the device-side error word
+ * that kernels set when one of their bounded waits gives up: SSM_OK if none
+ * did since the previous call, SSM_ERR_TIMEOUT otherwise.  Kernel waits are
+ * on shared-memory barriers that complete asynchronous copies, each limited
+ * to about 2 s of clock cycles, so a fault in the copy engine surfaces here
+ * instead of hanging the stream.
+ */
+ssm_status_t ssm_device_error_status(void *stream);
+
 #ifdef __cplusplus
 }
 #endif

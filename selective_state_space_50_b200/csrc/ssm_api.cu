@@ -10,6 +10,35 @@
 
 #include "ssm_internal.h"
 
+// The device error word (see ssm_device_error_status).
+__device__ int g_ssm_device_error = 0;
+
+namespace ssm {
+
+int *device_error_word() {
+    static int *addr[64] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (!addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_ssm_device_error) != cudaSuccess) return nullptr;
+        addr[dev] = static_cast<int *>(p);
+    }
+    return addr[dev];
+}
+
+cudaError_t read_and_clear_device_error(int *value, cudaStream_t stream) {
+    int *w = device_error_word();
+    if (!w) return cudaErrorInvalidDevice;
+    cudaError_t e = cudaMemcpyAsync(value, w, sizeof(int), cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    if (e == cudaSuccess && *value) e = cudaMemsetAsync(w, 0, sizeof(int), stream);
+    if (e == cudaSuccess && *value) e = cudaStreamSynchronize(stream);
+    return e;
+}
+
+}  // namespace ssm
+
 namespace {
 
 thread_local std::string g_last_error;
@@ -225,6 +254,14 @@ ssm_status_t ssm_selective_scan_bwd(const ssm_shape_t *shape, const void *u, con
     p.io_bf16 = shape->io_dtype == SSM_BF16; p.vec_ok = vec_ok;
     e = ssm::launch_bwd(p, st);
     if (e != cudaSuccess) return cuda_fail(e, "ssm_selective_scan_bwd launch");
+    return ok();
+}
+
+ssm_status_t ssm_device_error_status(void *stream) {
+    int v = 0;
+    cudaError_t e = ssm::read_and_clear_device_error(&v, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "ssm_device_error_status");
+    if (v) return fail(SSM_ERR_TIMEOUT, "a bounded wait inside a kernel gave up (code %d)", v);
     return ok();
 }
 

@@ -120,7 +120,7 @@ bwd_kernel(const BwdParams p) {
                 if (j + i >= W) break;
                 const bool ok = (i < n_in) && dd < p.dim;
                 const float r = dr[i] + bias;
-                const float dt = ok ? (p.softplus ? softplus(r) : r) : 0.f;
+                const float dt = ok ? (p.softplus ? softplus_fast(r) : r) : 0.f;
                 const float x = ok ? uu[i] : 0.f;
                 sDt[cc * WS + j + i] = dt;
                 sDu[cc * WS + j + i] = dt * x;

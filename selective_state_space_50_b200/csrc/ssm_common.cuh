@@ -16,14 +16,42 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
-// softplus(r) = log(1 + e^r).  Above r = 20, log1p(e^r) - r = log1p(e^-r) is
-// below 2.1e-9, under half an ulp of r in fp32, so r itself is returned.
-__device__ __forceinline__ float softplus(float r) {
-    return r > 20.f ? r : log1pf(__expf(r));
-}
-
 __device__ __forceinline__ float sigmoid(float v) {
     return __fdividef(1.f, 1.f + __expf(-v));
+}
+
+__device__ __forceinline__ float lg2(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ float tanh_approx(float x) {
+    float y;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// softplus(r) = ln(1 + e^r) from the hardware base-2 units:
+//   x = e^r = 2^(r log2 e);  ln(1 + x) = lg2(1 + x) ln 2  for x >= 1/32,
+//   and below that the Taylor series ln(1+x) = x - x^2/2 + x^3/3 - x^4/4
+//   (truncation error under x^5/5, i.e. relative 2e-7 at x = 1/32), which
+//   avoids the cancellation of 1 + x.  Above r = 15, ln(1 + e^r) - r < 3.1e-7
+//   is below half an ulp of r, so r is returned.
+__device__ __forceinline__ float softplus_fast(float r) {
+    const float x = ex2(r * SSM_LOG2E);
+    const float series = x * fmaf(x, fmaf(x, fmaf(x, -0.25f, 0.33333334f), -0.5f), 1.f);
+    const float viaLog = lg2(1.f + x) * 0.69314718f;
+    const float v = x < 0.03125f ? series : viaLog;
+    return r > 15.f ? r : v;
+}
+
+// SiLU gate z * sigmoid(z) with sigmoid(z) = (1 + tanh(z/2)) / 2 on the
+// hardware tanh (one SFU op; relative error of tanh.approx ~2^-11, below the
+// rounding of a bf16 result).
+__device__ __forceinline__ float silu_tanh(float z) {
+    const float hz = 0.5f * z;
+    return fmaf(hz, tanh_approx(hz), hz);
 }
 
 // ---- io element types -------------------------------------------------------

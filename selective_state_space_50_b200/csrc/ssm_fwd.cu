@@ -26,10 +26,26 @@
 //  * Steps past the end of the sequence are staged as Δ = 0, so they leave
 //    the state unchanged (Ā = 1, no input) and nothing is stored for them.
 
+#include <stdlib.h>
+#include <string.h>
+
 #include "ssm_common.cuh"
 #include "ssm_internal.h"
 
 namespace ssm {
+
+// SSM_FWD_KERNEL=general|tma|auto (default auto) selects the forward kernel:
+// "tma" fails with cudaErrorNotSupported where the TMA kernel does not apply.
+FwdKernel fwd_kernel_choice() {
+    static int cached = -1;
+    if (cached < 0) {
+        const char *e = getenv("SSM_FWD_KERNEL");
+        cached = (e && !strcmp(e, "general")) ? (int)FwdKernel::kGeneral
+                 : (e && !strcmp(e, "tma"))   ? (int)FwdKernel::kTma
+                                              : (int)FwdKernel::kAuto;
+    }
+    return (FwdKernel)cached;
+}
 
 template <typename T, int NT, int NS, int G, int TT>
 struct FwdSmem {
@@ -107,7 +123,7 @@ fwd_kernel(const FwdParams p) {
 #pragma unroll
                 for (int i = 0; i < V; ++i) {
                     float r = dr[i] + bias;
-                    float dt = p.softplus ? softplus(r) : r;
+                    float dt = p.softplus ? softplus_fast(r) : r;
                     dr[i] = (i < n_in) ? dt : 0.f;
                 }
             } else {
@@ -219,7 +235,8 @@ fwd_kernel(const FwdParams p) {
                     float yy = fmaf(Dd, sU[cc * RS + j + i], y[i]);
                     if (z) {
                         const float zz = sZ[cc * RS + j + i];
-                        yy *= zz * sigmoid(zz);
+                        if constexpr (sizeof(T) == 2) yy *= silu_tanh(zz);
+                        else yy *= zz * sigmoid(zz);
                     }
                     y[i] = yy;
                 }
@@ -278,6 +295,12 @@ static cudaError_t launch_fwd_t(const FwdParams &p, cudaStream_t stream) {
 }
 
 cudaError_t launch_fwd(const FwdParams &p, bool states_only, cudaStream_t stream) {
+    const FwdKernel choice = fwd_kernel_choice();
+    if (!states_only && choice != FwdKernel::kGeneral) {
+        cudaError_t e = cudaSuccess;
+        if (try_launch_fwd_tma(p, stream, &e)) return e;
+        if (choice == FwdKernel::kTma) return cudaErrorNotSupported;
+    }
     if (p.io_bf16)
         return states_only ? launch_fwd_t<__nv_bfloat16, 1>(p, stream)
                            : launch_fwd_t<__nv_bfloat16, 0>(p, stream);

@@ -1,0 +1,485 @@
+// Forward selective scan, TMA-fed persistent kernel for sm_100a.
+//
+// Same arithmetic as ssm_fwd.cu (booiljung.github.io "3.2 선택적 스캔(Selective
+// Scan) 알고리즘" §1.1/§1.2/§2.1, fused as in its §3.2): Δ = softplus(delta +
+// bias), Ā = exp(Δ A), h = Ā h + Δ B u, y = C·h + D u, out = y silu(z).
+//
+// Layout of the work:
+//  * One CTA per SM.  The batch*dim channel rows are split over the CTAs to
+//    within one row, so every SM does the same amount of work; a CTA may run
+//    its rows in several passes when they exceed one pass's capacity.
+//  * One producer lane streams fixed-size time tiles (TT steps) of delta, u,
+//    z (a [rows x TT] box each) and B, C (a [dstate x TT] box per batch row)
+//    into a STAGES-deep shared-memory ring with 2-D TMA loads completing on
+//    mbarriers.
+//  * Consumer warps own 32/NT channels each; lane (c, g) owns NS = N/NT
+//    states of channel c and keeps them in fp32 registers for the whole
+//    sequence.  Per tile a warp (1) computes Δ and Δ·u once per element into
+//    a warp-private fp32 buffer, (2) runs the recurrence, two time steps per
+//    f32x2 instruction and one ex2 per (step, state), reading B and C in the
+//    io dtype straight from the TMA tile (shared memory delivers at most 128
+//    bytes per clock per SM to the lanes, and B/C are re-read by every lane
+//    for every step, so their width sets the kernel's shared-memory time),
+//    and writes each lane's partial readout Σ_{own n} C h to shared memory,
+//    (3) sums the NT partials, applies D·u and the SiLU gate and writes y
+//    with 16-byte stores.  Warps synchronise only through the ring's
+//    mbarriers; every wait is bounded (kWaitBudgetCycles).
+
+#include <cudaTypedefs.h>
+
+#include <stdlib.h>
+
+#include <algorithm>
+
+#include "ssm_common.cuh"
+#include "ssm_internal.h"
+#include "ssm_tma.cuh"
+
+// Build-time tuning knobs (defaults are the measured best on B200).
+#ifndef SSM_TMA_STAGES
+#define SSM_TMA_STAGES 3      // depth of the TMA ring for bf16 io
+#endif
+#ifndef SSM_TMA_UNROLL
+#define SSM_TMA_UNROLL 2      // 8-step blocks unrolled in the recurrence loop
+#endif
+
+namespace ssm {
+
+namespace {
+
+constexpr int kTmaUnroll = SSM_TMA_UNROLL;
+
+constexpr int align128(int x) { return (x + 127) / 128 * 128; }
+
+struct TmaFwdParams {
+    const float *A, *D, *delta_bias;
+    void *out;
+    float *last_state, *ckpt;
+    int P;          // batch * dim channel rows
+    int dim, L, n_ckpt;
+    int softplus, has_z;
+    int rows_max;   // rows of one pass (= box height of the per-channel maps)
+    int *err;       // device error word
+};
+
+template <typename T, int NT, int NS, int TT, int NWC, int STAGES>
+struct TmaLayout {
+    static constexpr int N = NT * NS;
+    static constexpr int CPW = 32 / NT;            // channels per consumer warp
+    static constexpr int MAXR = NWC * CPW;         // rows per pass, at most
+    static constexpr int ES = sizeof(T);
+    static constexpr int RAW_ROW = TT * ES;
+    static constexpr int RAW_CH = align128(MAXR * RAW_ROW);
+    static constexpr int RAW_BC = align128(2 * N * RAW_ROW);   // up to two batch rows
+    static constexpr int STAGE = 3 * RAW_CH + 2 * RAW_BC;
+    static constexpr int WS = TT + 4;                          // fp32 row stride (floats)
+    static constexpr int WBUF = (2 + NT) * CPW * WS * 4;       // Δ, Δ·u, NT readout partials
+    static constexpr int kW = STAGES * STAGE;
+    static constexpr int kBar = kW + NWC * WBUF;
+    static constexpr int kTotal = kBar + 2 * STAGES * 8;
+    static constexpr int kThreads = (NWC + 1) * 32;
+    static constexpr int CHUNK = 8;                            // steps per prep/epilogue item
+    static constexpr int ITEMS = CPW * (TT / CHUNK);           // (row, chunk) items per warp
+    static_assert(kTotal <= 227 * 1024, "shared memory budget");
+    static_assert(TT % 8 == 0 && ITEMS % 32 == 0, "tile shape");
+    static_assert(NT == 2 || NT == 4 || NT == 8, "lane split");
+};
+
+// Loads 8 consecutive time steps of one B or C row from a raw stage tile
+// (io dtype) as four fp32 pairs {t, t+1}.
+template <typename T>
+__device__ __forceinline__ void load_pairs8(const T *src, float2 (&v)[4]);
+
+template <>
+__device__ __forceinline__ void load_pairs8<__nv_bfloat16>(const __nv_bfloat16 *src, float2 (&v)[4]) {
+    const uint4 q = *reinterpret_cast<const uint4 *>(src);
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        v[i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xffff0000u));
+}
+
+template <>
+__device__ __forceinline__ void load_pairs8<float>(const float *src, float2 (&v)[4]) {
+    const float4 a = *reinterpret_cast<const float4 *>(src);
+    const float4 b = *reinterpret_cast<const float4 *>(src + 4);
+    v[0] = make_float2(a.x, a.y); v[1] = make_float2(a.z, a.w);
+    v[2] = make_float2(b.x, b.y); v[3] = make_float2(b.z, b.w);
+}
+
+template <typename T, int NT, int NS, int TT, int NWC, int STAGES>
+__global__ void __launch_bounds__((NWC + 1) * 32, 1)
+fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constant__ CUtensorMap m_u,
+               const __grid_constant__ CUtensorMap m_z, const __grid_constant__ CUtensorMap m_B,
+               const __grid_constant__ CUtensorMap m_C, const TmaFwdParams p) {
+    using Ly = TmaLayout<T, NT, NS, TT, NWC, STAGES>;
+    constexpr int N = Ly::N, CPW = Ly::CPW, WS = Ly::WS, CHUNK = Ly::CHUNK;
+    constexpr int IPL = Ly::ITEMS / 32;   // prep/epilogue items per lane
+    constexpr int CPR = TT / CHUNK;       // chunks per row
+
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + Ly::kBar);
+    uint64_t *empty = full + STAGES;
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int G = gridDim.x;
+    const int r0 = (int)((long long)blockIdx.x * p.P / G);
+    const int r1 = (int)((long long)(blockIdx.x + 1) * p.P / G);
+    const int R = r1 - r0;
+    const int npass = (R + p.rows_max - 1) / p.rows_max;
+    const int ntiles = (p.L + TT - 1) / TT;
+    const int total = npass * ntiles;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(full + s, 1);
+            mbar_init(empty + s, NWC);
+        }
+        fence_barrier_init();
+    }
+    __syncthreads();
+
+    // rows of pass q: [q0, q1), split evenly
+    auto pass_rows = [&](int q, int &q0, int &q1) {
+        q0 = r0 + (int)((long long)q * R / npass);
+        q1 = r0 + (int)((long long)(q + 1) * R / npass);
+    };
+
+    if (warp == NWC) {
+        // ------------------------------------------------------------ producer
+        if (lane != 0) return;
+        prefetch_tensormap(&m_delta);
+        prefetch_tensormap(&m_u);
+        if (p.has_z) prefetch_tensormap(&m_z);
+        prefetch_tensormap(&m_B);
+        prefetch_tensormap(&m_C);
+        int issued = 0;
+        bool ok = true;
+        int s = 0, phase = 0, q = 0, tile = 0, q0 = 0, q1 = 0, b_lo = 0, nb = 1;
+        for (; issued < total && ok; ++issued) {
+            if (issued >= STAGES) {   // wait until every consumer left this stage
+                ok = mbar_wait(empty + s, phase ^ 1, p.err);
+                if (!ok) break;
+            }
+            if (tile == 0) {
+                pass_rows(q, q0, q1);
+                b_lo = q0 / p.dim;
+                nb = (q1 - 1) / p.dim - b_lo + 1;
+            }
+            const int t0 = tile * TT;
+            uint8_t *st = smem + s * Ly::STAGE;
+            const uint32_t bytes = (uint32_t)(p.rows_max * Ly::RAW_ROW * (2 + p.has_z) +
+                                              2 * nb * N * Ly::RAW_ROW);
+            mbar_arrive_expect_tx(full + s, bytes);
+            tma_load_2d(st, &m_delta, t0, q0, full + s);
+            tma_load_2d(st + Ly::RAW_CH, &m_u, t0, q0, full + s);
+            if (p.has_z) tma_load_2d(st + 2 * Ly::RAW_CH, &m_z, t0, q0, full + s);
+            for (int bs = 0; bs < nb; ++bs) {
+                tma_load_2d(st + 3 * Ly::RAW_CH + bs * N * Ly::RAW_ROW, &m_B, t0, (b_lo + bs) * N, full + s);
+                tma_load_2d(st + 3 * Ly::RAW_CH + Ly::RAW_BC + bs * N * Ly::RAW_ROW, &m_C, t0,
+                            (b_lo + bs) * N, full + s);
+            }
+            if (++s == STAGES) { s = 0; phase ^= 1; }
+            if (++tile == ntiles) { tile = 0; ++q; }
+        }
+        // Never leave while a copy may still write shared memory: the last
+        // STAGES loads are the only ones no consumer is known to have seen.
+        for (int kg = (issued > STAGES ? issued - STAGES : 0); kg < issued; ++kg)
+            if (!mbar_wait(full + (kg % STAGES), (kg / STAGES) & 1, p.err)) break;
+        return;
+    }
+
+    // ---------------------------------------------------------------- consumers
+    // Scan mapping: lane = g * CPW + c (a quarter-warp shares one state group,
+    // so its B/C reads are one broadcast row).  Prep/epilogue mapping: item
+    // lane + 32 i = (row, 8-step chunk), contiguous in shared memory.
+    const int c = lane % CPW, g = lane / CPW;
+    float *wDt = reinterpret_cast<float *>(smem + Ly::kW + warp * Ly::WBUF);
+    float *wDu = wDt + CPW * WS;
+    float *wY = wDu + CPW * WS;      // [NT][CPW][WS] readout partials
+
+    float2 A2d[NS];                  // A[d, n] log2(e), duplicated for f32x2 math
+    float h[NS];
+    int bsel = 0;
+    bool live = false;
+    // per-item constants for the prep / epilogue rows
+    float Dd[IPL], bias[IPL];
+    int irow[IPL];
+
+    int s = 0, phase = 0;          // ring slot and its parity for tile kg
+    int q = 0, tile = 0, q0 = 0, q1 = 0;
+    for (int kg = 0; kg < total; ++kg) {
+        if (tile == 0) pass_rows(q, q0, q1);
+        const int t0 = tile * TT;
+        const int wrow0 = q0 + warp * CPW;   // first row of this warp in the pass
+        if (tile == 0) {
+            const int row = wrow0 + c;
+            live = row < q1;
+            const int d = live ? row % p.dim : 0;
+            bsel = live ? row / p.dim - q0 / p.dim : 0;
+#pragma unroll
+            for (int j = 0; j < NS; ++j) {
+                const float a = live ? p.A[(size_t)d * N + g * NS + j] * SSM_LOG2E : 0.f;
+                A2d[j] = make_float2(a, a);
+                h[j] = 0.f;
+            }
+#pragma unroll
+            for (int i = 0; i < IPL; ++i) {
+                const int rr = wrow0 + (lane + 32 * i) / CPR;
+                const bool ok = rr < q1;
+                const int dd = ok ? rr % p.dim : 0;
+                irow[i] = ok ? rr : -1;
+                Dd[i] = (ok && p.D) ? p.D[dd] : 0.f;
+                bias[i] = (ok && p.delta_bias) ? p.delta_bias[dd] : 0.f;
+            }
+        }
+        if (!mbar_wait(full + s, phase, p.err)) return;
+
+        if (wrow0 < q1) {
+            const uint8_t *st = smem + s * Ly::STAGE;
+            const T *rawD = reinterpret_cast<const T *>(st) + warp * CPW * TT;
+            const T *rawU = reinterpret_cast<const T *>(st + Ly::RAW_CH) + warp * CPW * TT;
+            const T *rawZ = reinterpret_cast<const T *>(st + 2 * Ly::RAW_CH) + warp * CPW * TT;
+            // (1) Δ and Δ·u, once per element
+#pragma unroll
+            for (int i = 0; i < IPL; ++i) {
+                const int it = lane + 32 * i, rl = it / CPR, t = (it % CPR) * CHUNK;
+                float dt[CHUNK], du[CHUNK];
+#pragma unroll
+                for (int v0 = 0; v0 < CHUNK; v0 += IO<T>::kVec) {
+                    constexpr int V = IO<T>::kVec;
+                    float dr[V], uu[V];
+                    IO<T>::unpack(*reinterpret_cast<const uint4 *>(rawD + rl * TT + t + v0), dr);
+                    IO<T>::unpack(*reinterpret_cast<const uint4 *>(rawU + rl * TT + t + v0), uu);
+#pragma unroll
+                    for (int k = 0; k < V; ++k) {
+                        const float r = dr[k] + bias[i];
+                        const bool ok = irow[i] >= 0 && (t0 + t + v0 + k) < p.L;
+                        dt[v0 + k] = ok ? (p.softplus ? softplus_fast(r) : r) : 0.f;
+                        du[v0 + k] = dt[v0 + k] * uu[k];
+                    }
+                }
+#pragma unroll
+                for (int k = 0; k < CHUNK; k += 4) {
+                    *reinterpret_cast<float4 *>(wDt + rl * WS + t + k) = make_float4(dt[k], dt[k + 1], dt[k + 2], dt[k + 3]);
+                    *reinterpret_cast<float4 *>(wDu + rl * WS + t + k) = make_float4(du[k], du[k + 1], du[k + 2], du[k + 3]);
+                }
+            }
+            __syncwarp();
+            // (2) the recurrence, two time steps per f32x2 op; B and C are read
+            // in the io dtype straight from the TMA tile
+            const T *rawB = reinterpret_cast<const T *>(st + 3 * Ly::RAW_CH) + (bsel * N + g * NS) * TT;
+            const T *rawC = reinterpret_cast<const T *>(st + 3 * Ly::RAW_CH + Ly::RAW_BC) + (bsel * N + g * NS) * TT;
+            float *myY = wY + (g * CPW + c) * WS;
+#pragma unroll kTmaUnroll
+            for (int tb = 0; tb < TT; tb += 8) {
+                float2 dtp[4], dup[4];
+                {
+                    const float4 a = *reinterpret_cast<const float4 *>(wDt + c * WS + tb);
+                    const float4 b = *reinterpret_cast<const float4 *>(wDt + c * WS + tb + 4);
+                    const float4 e = *reinterpret_cast<const float4 *>(wDu + c * WS + tb);
+                    const float4 f = *reinterpret_cast<const float4 *>(wDu + c * WS + tb + 4);
+                    dtp[0] = make_float2(a.x, a.y); dtp[1] = make_float2(a.z, a.w);
+                    dtp[2] = make_float2(b.x, b.y); dtp[3] = make_float2(b.z, b.w);
+                    dup[0] = make_float2(e.x, e.y); dup[1] = make_float2(e.z, e.w);
+                    dup[2] = make_float2(f.x, f.y); dup[3] = make_float2(f.z, f.w);
+                }
+                float2 y2[4];
+#pragma unroll
+                for (int pp = 0; pp < 4; ++pp) y2[pp] = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int j = 0; j < NS; ++j) {
+                    float2 bq[4], cq[4];
+                    load_pairs8<T>(rawB + j * TT + tb, bq);
+                    load_pairs8<T>(rawC + j * TT + tb, cq);
+#pragma unroll
+                    for (int pp = 0; pp < 4; ++pp) {
+                        const float2 arg = __fmul2_rn(dtp[pp], A2d[j]);
+                        const float a0 = ex2(arg.x), a1 = ex2(arg.y);
+                        const float2 beta = __fmul2_rn(dup[pp], bq[pp]);
+                        const float h0 = fmaf(a0, h[j], beta.x);
+                        const float h1 = fmaf(a1, h0, beta.y);
+                        h[j] = h1;
+                        y2[pp] = __ffma2_rn(cq[pp], make_float2(h0, h1), y2[pp]);
+                    }
+                }
+                *reinterpret_cast<float4 *>(myY + tb) = make_float4(y2[0].x, y2[0].y, y2[1].x, y2[1].y);
+                *reinterpret_cast<float4 *>(myY + tb + 4) = make_float4(y2[2].x, y2[2].y, y2[3].x, y2[3].y);
+            }
+            // checkpoints and the final state
+            const int tend = min(t0 + TT, p.L);
+            const int row = wrow0 + c;
+            if (live && p.ckpt && (tend % SSM_CKPT_CHUNK == 0 || tend == p.L)) {
+                float *dst = p.ckpt + ((size_t)row * p.n_ckpt + (tend - 1) / SSM_CKPT_CHUNK) * N + g * NS;
+#pragma unroll
+                for (int j = 0; j < NS; ++j) dst[j] = h[j];
+            }
+            if (live && p.last_state && tile == ntiles - 1) {
+                float *dst = p.last_state + (size_t)row * N + g * NS;
+#pragma unroll
+                for (int j = 0; j < NS; ++j) dst[j] = h[j];
+            }
+            __syncwarp();
+            // (3) Σ of the NT partials, D skip, gate, 16-byte stores
+#pragma unroll
+            for (int i = 0; i < IPL; ++i) {
+                const int it = lane + 32 * i, rl = it / CPR, t = (it % CPR) * CHUNK;
+                if (irow[i] < 0 || t0 + t >= p.L) continue;
+                float y[CHUNK];
+#pragma unroll
+                for (int k = 0; k < CHUNK; k += 4) {
+                    float2 lo = make_float2(0.f, 0.f), hi = make_float2(0.f, 0.f);
+#pragma unroll
+                    for (int gg = 0; gg < NT; ++gg) {
+                        const float4 q4 = *reinterpret_cast<const float4 *>(wY + (gg * CPW + rl) * WS + t + k);
+                        lo = __fadd2_rn(lo, make_float2(q4.x, q4.y));
+                        hi = __fadd2_rn(hi, make_float2(q4.z, q4.w));
+                    }
+                    y[k] = lo.x; y[k + 1] = lo.y; y[k + 2] = hi.x; y[k + 3] = hi.y;
+                }
+                T *out = static_cast<T *>(p.out) + (size_t)irow[i] * p.L + t0 + t;
+#pragma unroll
+                for (int v0 = 0; v0 < CHUNK; v0 += IO<T>::kVec) {
+                    constexpr int V = IO<T>::kVec;
+                    float uu[V], zz[V], o[V];
+                    IO<T>::unpack(*reinterpret_cast<const uint4 *>(rawU + rl * TT + t + v0), uu);
+                    if (p.has_z) IO<T>::unpack(*reinterpret_cast<const uint4 *>(rawZ + rl * TT + t + v0), zz);
+#pragma unroll
+                    for (int k = 0; k < V; ++k) {
+                        float yy = fmaf(Dd[i], uu[k], y[v0 + k]);
+                        if (p.has_z) {
+                            if constexpr (sizeof(T) == 2) yy *= silu_tanh(zz[k]);
+                            else yy *= zz[k] * sigmoid(zz[k]);
+                        }
+                        o[k] = yy;
+                    }
+                    __stcs(reinterpret_cast<uint4 *>(out + v0), IO<T>::pack(o));
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty + s);
+        if (++s == STAGES) { s = 0; phase ^= 1; }
+        if (++tile == ntiles) { tile = 0; ++q; }
+    }
+}
+
+// ------------------------------------------------------------------ host side
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+bool make_map(CUtensorMap *m, const void *base, bool bf16, uint64_t rows, uint64_t cols, uint32_t box_cols,
+              uint32_t box_rows) {
+    auto enc = get_encode();
+    if (!enc) return false;
+    const uint64_t es = bf16 ? 2 : 4;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * es};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+                     const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int sm_count() {
+    static int count[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) return 148;
+    if (!count[dev]) cudaDeviceGetAttribute(&count[dev], cudaDevAttrMultiProcessorCount, dev);
+    return count[dev];
+}
+
+template <typename T, int NT, int NS, int TT, int NWC, int STAGES>
+cudaError_t launch_cfg(const FwdParams &fp, cudaStream_t stream) {
+    using Ly = TmaLayout<T, NT, NS, TT, NWC, STAGES>;
+    const int P = fp.batch * fp.dim;
+    const int grid = std::min(sm_count(), P);
+    const int R = (P + grid - 1) / grid;
+    const int npass = (R + Ly::MAXR - 1) / Ly::MAXR;
+    const int rows_max = (R + npass - 1) / npass;
+    const bool bf16 = sizeof(T) == 2;
+    CUtensorMap md, mu, mz, mB, mC;
+    if (!make_map(&md, fp.delta, bf16, P, fp.L, TT, rows_max) ||
+        !make_map(&mu, fp.u, bf16, P, fp.L, TT, rows_max) ||
+        !make_map(&mz, fp.z ? fp.z : fp.u, bf16, P, fp.L, TT, rows_max) ||
+        !make_map(&mB, fp.B, bf16, (uint64_t)fp.batch * fp.N, fp.L, TT, Ly::N) ||
+        !make_map(&mC, fp.C, bf16, (uint64_t)fp.batch * fp.N, fp.L, TT, Ly::N))
+        return cudaErrorInvalidValue;
+    TmaFwdParams p{};
+    p.A = fp.A; p.D = fp.D; p.delta_bias = fp.delta_bias; p.out = fp.out;
+    p.last_state = fp.last_state; p.ckpt = fp.ckpt;
+    p.P = P; p.dim = fp.dim; p.L = fp.L; p.n_ckpt = fp.n_ckpt;
+    p.softplus = fp.softplus; p.has_z = fp.z != nullptr; p.rows_max = rows_max;
+    p.err = device_error_word();
+    if (!p.err) return cudaErrorInvalidDevice;
+    auto kern = fwd_tma_kernel<T, NT, NS, TT, NWC, STAGES>;
+    static bool attr_done = false;
+    if (!attr_done) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Ly::kTotal);
+        if (e != cudaSuccess) return e;
+        attr_done = true;
+    }
+    kern<<<grid, Ly::kThreads, Ly::kTotal, stream>>>(md, mu, mz, mB, mC, p);
+    return cudaGetLastError();
+}
+
+// Consumer warps per CTA for each lane split and io width (as many as the
+// shared-memory budget allows), and the rows one pass of it holds.
+constexpr int nwc_for(int nt, bool bf16) { return bf16 ? (nt == 4 ? 12 : 9) : 8; }
+constexpr int rows_cap(int nt, bool bf16) { return nwc_for(nt, bf16) * (32 / nt); }
+
+}  // namespace
+
+// Returns true (and launches) when the TMA path applies; false means the
+// caller should use the general kernel.
+bool try_launch_fwd_tma(const FwdParams &fp, cudaStream_t stream, cudaError_t *err) {
+    if (!fp.vec_ok || !fp.out) return false;
+    if (fp.N != 8 && fp.N != 16 && fp.N != 32) return false;
+    if (!get_encode()) return false;
+    const long long P = (long long)fp.batch * fp.dim;
+    const int sms = sm_count();
+    if (P < 32LL * sms) return false;               // too few channels: not enough lanes
+    const long long R = (P + sms - 1) / sms;
+    // choose the lane split: 4 lanes per channel while one pass holds the rows
+    int nt = (fp.N == 8) ? 2 : (fp.N == 32 ? 4 : (R <= rows_cap(4, fp.io_bf16) ? 4 : 2));
+    // SSM_TMA_NT=2|4 overrides the lane split for dstate 16 (tuning knob)
+    static const char *force_nt = getenv("SSM_TMA_NT");
+    if (fp.N == 16 && force_nt && (force_nt[0] == '2' || force_nt[0] == '4')) nt = force_nt[0] - '0';
+    const long long cap = rows_cap(nt, fp.io_bf16);
+    const long long npass = (R + cap - 1) / cap;
+    const long long rows_pass = (R + npass - 1) / npass;
+    if (rows_pass > fp.dim) return false;           // a pass may touch at most two batch rows
+    cudaError_t e;
+    if (fp.io_bf16) {
+        using T = __nv_bfloat16;
+        if (fp.N == 8) e = launch_cfg<T, 2, 4, 32, nwc_for(2, true), SSM_TMA_STAGES>(fp, stream);
+        else if (fp.N == 16) e = nt == 4 ? launch_cfg<T, 4, 4, 32, nwc_for(4, true), SSM_TMA_STAGES>(fp, stream)
+                                         : launch_cfg<T, 2, 8, 32, nwc_for(2, true), SSM_TMA_STAGES>(fp, stream);
+        else e = launch_cfg<T, 4, 8, 32, nwc_for(4, true), SSM_TMA_STAGES>(fp, stream);
+    } else {
+        using T = float;
+        if (fp.N == 8) e = launch_cfg<T, 2, 4, 32, nwc_for(2, false), 2>(fp, stream);
+        else if (fp.N == 16) e = nt == 4 ? launch_cfg<T, 4, 4, 32, nwc_for(4, false), 2>(fp, stream)
+                                         : launch_cfg<T, 2, 8, 32, nwc_for(2, false), 2>(fp, stream);
+        else e = launch_cfg<T, 4, 8, 32, nwc_for(4, false), 2>(fp, stream);
+    }
+    *err = e;
+    return true;
+}
+
+}  // namespace ssm

@@ -38,7 +38,19 @@ struct BwdParams {
     bool vec_ok;
 };
 
+enum class FwdKernel { kAuto = 0, kGeneral = 1, kTma = 2 };
+FwdKernel fwd_kernel_choice();
+
 cudaError_t launch_fwd(const FwdParams &p, bool states_only, cudaStream_t stream);
+// Launches the TMA-fed persistent forward when it applies (returns true and
+// sets *err); returns false when the general kernel must be used.
+bool try_launch_fwd_tma(const FwdParams &p, cudaStream_t stream, cudaError_t *err);
+// Device address of the error word that kernels set when a bounded wait
+// gives up (one word per device, looked up once per device); NULL on failure.
+int *device_error_word();
+// Copies the device error word to *value (after synchronising `stream`) and
+// clears it when set.
+cudaError_t read_and_clear_device_error(int *value, cudaStream_t stream);
 cudaError_t launch_bwd(const BwdParams &p, cudaStream_t stream);
 
 }  // namespace ssm

@@ -14,7 +14,9 @@ from typing import Optional
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libssmscan.so")
+# SSM_LIB_PATH selects another build of the library (e.g. one compiled with
+# different tuning macros); the default is the in-tree build.
+LIB_PATH = os.environ.get("SSM_LIB_PATH") or os.path.join(_HERE, "libssmscan.so")
 
 SSM_OK, SSM_ERR_INVALID_ARG, SSM_ERR_UNSUPPORTED, SSM_ERR_CUDA, SSM_ERR_TIMEOUT = range(5)
 SSM_F32, SSM_BF16 = 0, 1
@@ -22,7 +24,7 @@ CKPT_CHUNK = 64  # SSM_CKPT_CHUNK in include/ssm_scan.h
 
 EXPORTS = ("ssm_version", "ssm_last_error_string", "ssm_selective_scan_ckpt_bytes",
            "ssm_selective_scan_fwd", "ssm_selective_scan_bwd_scratch_bytes",
-           "ssm_selective_scan_bwd")
+           "ssm_selective_scan_bwd", "ssm_device_error_status")
 
 
 class SSMError(RuntimeError):
@@ -60,12 +62,19 @@ def load_library(path: str = LIB_PATH):
     lib.ssm_selective_scan_fwd.restype = i
     lib.ssm_selective_scan_bwd.argtypes = [sp] + [vp] * 8 + [i] + [vp] * 11 + [sz, vp]
     lib.ssm_selective_scan_bwd.restype = i
+    lib.ssm_device_error_status.argtypes = [vp]
+    lib.ssm_device_error_status.restype = i
     _lib = lib
     return lib
 
 
 def last_error() -> str:
     return load_library().ssm_last_error_string().decode()
+
+
+def device_error_status(stream=None):
+    """Synchronises the stream and raises SSMError if a kernel's bounded wait gave up."""
+    _check(load_library().ssm_device_error_status(_stream_ptr(stream)))
 
 
 def _check(status: int):

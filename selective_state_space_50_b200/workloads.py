@@ -142,7 +142,7 @@ class Workload:
     softplus: bool = True
     D_dist: str = "ones"     # "ones" | "u0.5_1.5"
     A_dist: str = "neg_n1"   # "neg_n1": A[d,n] = -(n+1); "neg_lognormal": -exp(N(0,1))
-    bias_dist: str = "expm1_u"   # "expm1_u": log(expm1(U[1e-3, 0.1])); "long_memory"
+    bias_dist: str = "expm1_u"   # "expm1_u": log(expm1(U[1e-3, 0.1])); "long_memory"; "step_u"
     delta_std: float = 1.0
     delta_abs: bool = False  # |N(0, std)| raw deltas (for callers passing Δ without softplus)
 
@@ -200,7 +200,11 @@ def generate(w: Workload, with_dout: bool = False,
         out[name + "_f64"] = f.astype(np.float64)
 
     # delta_bias
-    if w.bias_dist == "expm1_u":
+    if w.bias_dist == "step_u":
+        # the bias is itself a step size in [1e-3, 0.1] (no softplus applied)
+        put32("delta_bias", uniform(w.seed, STREAMS["delta_bias"], Dm, 1e-3, 0.1))
+        d0 = None
+    elif w.bias_dist == "expm1_u":
         d0 = uniform(w.seed, STREAMS["delta_bias"], Dm, 1e-3, 0.1)
     elif w.bias_dist == "long_memory":
         # log-uniform step size in [1.5e-4, 4.5e-3]
@@ -208,7 +212,8 @@ def generate(w: Workload, with_dout: bool = False,
                             math.log(1.5e-4), math.log(4.5e-3)))
     else:
         raise ValueError(w.bias_dist)
-    put32("delta_bias", np.log(np.expm1(d0)))
+    if d0 is not None:
+        put32("delta_bias", np.log(np.expm1(d0)))
 
     if w.D_dist == "ones":
         put32("D", np.ones(Dm))

@@ -84,7 +84,8 @@ def small_workload(batch, dim, L, N, io, z, D, bias, sp, A_dist, seed=77):
     # (a negative step makes Ā > 1 and the state grows without bound)
     return Workload("small", batch, L, dim, N, io, seed=seed, has_z=z, has_D=D, has_bias=bias,
                     softplus=sp, A_dist=A_dist, D_dist="u0.5_1.5",
-                    delta_abs=not sp, delta_std=1.0 if sp else 0.1)
+                    delta_abs=not sp, delta_std=1.0 if sp else 0.1,
+                    bias_dist="expm1_u" if sp else "step_u")
 
 
 @pytest.mark.parametrize("case", SMALL)
@@ -185,3 +186,85 @@ def test_bwd_small(case, use_ckpt):
 
 def test_bwd_layer_shape_full():
     check_bwd(WORKLOADS["mamba130m_layer_fwdbwd"], use_ckpt=True)
+
+
+# ------------------------------------------------------------------ TMA forward path
+# Shapes with >= 32 channels per SM and L a multiple of 8 take the TMA-fed
+# persistent kernel; these cover its ragged last tile, fp32 io, N = 8 / 32,
+# several passes per CTA and CTAs whose rows span two batch rows.
+TMA_CASES = [
+    # batch, dim, L, N, io, z, D, bias, softplus, A_dist
+    (2, 2400, 72, 16, "bf16", True, True, True, True, "neg_lognormal"),
+    (3, 2000, 40, 16, "f32", True, False, True, True, "neg_lognormal"),
+    (2, 2400, 64, 8, "bf16", False, True, False, True, "neg_lognormal"),
+    (2, 2400, 48, 32, "bf16", True, True, True, False, "neg_lognormal"),
+    (2, 15000, 16, 16, "bf16", True, True, True, True, "neg_lognormal"),
+    (4, 5120, 24, 16, "bf16", True, True, True, True, "neg_lognormal"),
+    (1, 4800, 1000, 16, "bf16", True, True, True, True, "neg_n1"),
+    (2, 3000, 200, 16, "f32", False, False, False, True, "neg_lognormal"),
+]
+
+
+@pytest.mark.parametrize("case", TMA_CASES)
+def test_fwd_tma_path(case):
+    check_fwd(small_workload(*case))
+
+
+def test_fwd_tma_ckpt_and_state():
+    w = small_workload(2, 2400, 136, 16, "bf16", True, True, True, True, "neg_lognormal")
+    inp = generate(w)
+    dv = to_device(inp, w)
+    out, last, ck = run_fwd(dv, w, return_ckpt=True)
+    ck = to_f64(ck).reshape(2, 2400, -1, 16)
+    chans = slice(0, 2400, 37)
+    sub = subset_channels(inp, chans)
+    for k in range(ck.shape[2]):
+        tend = min(136, (k + 1) * ssm_scan.CKPT_CHUNK)
+        _, st = oracle.fwd(sub["u_f64"][..., :tend], sub["delta_f64"][..., :tend], sub["A_f64"],
+                           sub["B_f64"][..., :tend], sub["C_f64"][..., :tend], sub["D_f64"],
+                           sub["z_f64"][..., :tend], sub["delta_bias_f64"], True)
+        assert_close_io(ck[:, chans, k], st, "bf16", f"ckpt[{k}]")
+
+
+def _run_forced(kernel, shape_args):
+    """Runs one forward in a fresh process with SSM_FWD_KERNEL set; returns its
+    stdout (the kernel choice is read once per process)."""
+    import os
+    import subprocess
+    import sys
+    code = (
+        "import sys; sys.path.insert(0, %r); sys.path.insert(0, %r)\n"
+        "import torch, numpy as np, oracle\n"
+        "from selective_state_space_50_b200 import ssm_scan\n"
+        "from selective_state_space_50_b200.workloads import Workload, generate, to_torch\n"
+        "w = Workload('f', *%r, seed=5, A_dist='neg_lognormal', D_dist='u0.5_1.5')\n"
+        "inp = generate(w); dv = to_torch(inp, w, 'cuda')\n"
+        "try:\n"
+        "    out, _, _ = ssm_scan.selective_scan_fwd(dv['u'], dv['delta'], dv['A'], dv['B'], dv['C'],"
+        " dv['D'], dv['z'], dv['delta_bias'], True)\n"
+        "    torch.cuda.synchronize()\n"
+        "except ssm_scan.SSMError as e:\n"
+        "    print('SSMError', e.status); raise SystemExit(0)\n"
+        "ref, _ = oracle.fwd_workload(inp, w)\n"
+        "err = np.abs(out.float().cpu().double().numpy() - ref) / (1 + np.abs(ref))\n"
+        "print('maxerr', err.max())\n"
+    ) % (os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+         os.path.dirname(os.path.abspath(__file__)), shape_args)
+    env = dict(os.environ, SSM_FWD_KERNEL=kernel)
+    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True,
+                       timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    return r.stdout
+
+
+def test_forced_kernel_selection():
+    # batch, seqlen, dim, dstate, io
+    big = (2, 64, 2400, 16, "bf16")
+    small = (1, 64, 40, 16, "bf16")
+    for kern in ("tma", "general"):
+        outp = _run_forced(kern, big)
+        assert "maxerr" in outp and float(outp.split()[-1]) <= 2e-2, outp
+    # the TMA kernel refuses shapes it does not cover
+    assert "SSMError 3" in _run_forced("tma", small)
+    outp = _run_forced("general", small)
+    assert float(outp.split()[-1]) <= 2e-2
