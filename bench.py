@@ -223,13 +223,13 @@ def run_ours(args, world, rank, local):
     from selective_state_space_50_b200 import ssm_scan
     from selective_state_space_50_b200.workloads import WORKLOADS, generate, to_torch
 
-    w = WORKLOADS[WORKLOAD]
+    w = WORKLOADS[args.workload]
     dev = torch.device("cuda", local)
     # every rank processes its own batch of the same shape (weak scaling)
     w_rank = w.replace(seed=w.seed + 7919 * rank)
     inp = generate(w_rank)
     dv = to_torch(inp, w_rank, dev)
-    shape = ssm_scan.make_shape(w.batch, w.dim, w.seqlen, w.dstate, torch.bfloat16)
+    shape = ssm_scan.make_shape(w.batch, w.dim, w.seqlen, w.dstate, dv["u"].dtype)
     out = torch.empty_like(dv["u"])
     last = torch.empty(w.batch, w.dim, w.dstate, device=dev, dtype=torch.float32)
     stream = torch.cuda.current_stream(dev)
@@ -300,19 +300,19 @@ def run_ours(args, world, rank, local):
     sm_max = float(peaks.get("sm_max_mhz") or 1965.0)
     mufu_peak = SM_COUNT_B200 * MUFU_EX2_PER_CLK_PER_SM * sm_max * 1e6
     achieved = ex2 / mean_s
-    alg_bytes = algorithmic_bytes(w, 2)
+    alg_bytes = algorithmic_bytes(w, 2 if w.io_dtype == "bf16" else 4)
     traffic = None
     tp = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(tp):
         with open(tp) as f:
-            traffic = json.load(f).get("ssm_fwd_" + WORKLOAD)
+            traffic = json.load(f).get("ssm_fwd_" + w.name)
     line = {
         "metric": METRIC, "value": elems_all / t_max, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": max(3, args.warmup),
         "ms_per_step": t_max / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "dim": w.dim,
-                   "dstate": w.dstate, "io_dtype": "bf16", "state_dtype": "f32",
+                   "dstate": w.dstate, "io_dtype": w.io_dtype, "state_dtype": "f32",
                    "parallelism": f"replicas x{world} (independent batches)",
                    "l2": "flushed between steps (256 MiB write, outside the timed events)"},
         "gbs": alg_bytes / mean_s / 1e9,
@@ -343,6 +343,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--workload", default=WORKLOAD,
+                    help="workload to time (default: the Mamba-130M layer shape)")
     args = ap.parse_args()
     world, rank, local = dist_setup(args)
     try:

@@ -46,12 +46,60 @@ __device__ __forceinline__ float softplus_fast(float r) {
     return r > 15.f ? r : v;
 }
 
+// softplus_fast on a pair of values, with the polynomial and scalings in
+// f32x2 arithmetic.
+__device__ __forceinline__ float2 softplus_fast2(float2 r) {
+    const float2 a = __fmul2_rn(r, make_float2(SSM_LOG2E, SSM_LOG2E));
+    const float2 x = make_float2(ex2(a.x), ex2(a.y));
+    float2 s = __ffma2_rn(x, make_float2(-0.25f, -0.25f), make_float2(0.33333334f, 0.33333334f));
+    s = __ffma2_rn(x, s, make_float2(-0.5f, -0.5f));
+    s = __ffma2_rn(x, s, make_float2(1.f, 1.f));
+    s = __fmul2_rn(x, s);
+    const float2 one_x = __fadd2_rn(x, make_float2(1.f, 1.f));
+    const float2 lv = __fmul2_rn(make_float2(lg2(one_x.x), lg2(one_x.y)),
+                                 make_float2(0.69314718f, 0.69314718f));
+    float2 v;
+    v.x = r.x > 15.f ? r.x : (x.x < 0.03125f ? s.x : lv.x);
+    v.y = r.y > 15.f ? r.y : (x.y < 0.03125f ? s.y : lv.y);
+    return v;
+}
+
 // SiLU gate z * sigmoid(z) with sigmoid(z) = (1 + tanh(z/2)) / 2 on the
 // hardware tanh (one SFU op; relative error of tanh.approx ~2^-11, below the
 // rounding of a bf16 result).
 __device__ __forceinline__ float silu_tanh(float z) {
     const float hz = 0.5f * z;
     return fmaf(hz, tanh_approx(hz), hz);
+}
+
+__device__ __forceinline__ float2 silu_tanh2(float2 z) {
+    const float2 hz = __fmul2_rn(z, make_float2(0.5f, 0.5f));
+    return __ffma2_rn(hz, make_float2(tanh_approx(hz.x), tanh_approx(hz.y)), hz);
+}
+
+// 2^x for a pair of x <= 0 on the FMA pipe (no SFU op), for offloading part of
+// the discretisation's exponentials from the SFU.  Method: Cody-Waite style
+// range reduction x = j + r with j = round(x) (adding 1.5 * 2^23 rounds to an
+// integer held in the low mantissa bits), r in [-1/2, 1/2]; 2^r from a degree-5
+// polynomial fitted for minimax relative error on [-1/2, 1/2] (Lawson's
+// iteration, constant term fixed at 1; max relative error 2.4e-7 = 2^-22.0
+// when evaluated in fp32 Horner form); 2^j applied by adding j to the
+// exponent field.  Inputs below -126 are clamped (2^-126 ~ 1.2e-38 instead of
+// 0).  Valid for x <= 0 only: callers check that A <= 0.
+__device__ __forceinline__ float2 ex2_poly2(float2 x) {
+    x.x = fmaxf(x.x, -126.f);
+    x.y = fmaxf(x.y, -126.f);
+    const float2 t = __fadd2_rn(x, make_float2(12582912.f, 12582912.f));
+    const float2 j = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
+    const float2 r = __ffma2_rn(j, make_float2(-1.f, -1.f), x);
+    float2 p = __ffma2_rn(make_float2(0.0013276467f, 0.0013276467f), r,
+                          make_float2(0.009675542f, 0.009675542f));
+    p = __ffma2_rn(p, r, make_float2(0.055507135f, 0.055507135f));
+    p = __ffma2_rn(p, r, make_float2(0.2402212f, 0.2402212f));
+    p = __ffma2_rn(p, r, make_float2(0.69314694f, 0.69314694f));
+    p = __ffma2_rn(p, r, make_float2(1.f, 1.f));
+    return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                       __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
 
 // ---- io element types -------------------------------------------------------

@@ -16,11 +16,13 @@
 //    states of channel c and keeps them in fp32 registers for the whole
 //    sequence.  Per tile a warp (1) computes Δ and Δ·u once per element into
 //    a warp-private fp32 buffer, (2) runs the recurrence, two time steps per
-//    f32x2 instruction and one ex2 per (step, state), reading B and C in the
-//    io dtype straight from the TMA tile (shared memory delivers at most 128
-//    bytes per clock per SM to the lanes, and B/C are re-read by every lane
-//    for every step, so their width sets the kernel's shared-memory time),
-//    and writes each lane's partial readout Σ_{own n} C h to shared memory,
+//    f32x2 instruction and one ex2 per (step, state).  Lanes are numbered
+//    state-group-major, so the eight lanes of a quarter-warp read the same
+//    B/C row: a broadcast 16-byte shared load.  B and C stay in the io dtype
+//    (converted in registers): the SFU is fed through the same MIO queue as
+//    shared-memory instructions, so halving the B/C load count matters more
+//    than the conversion ALU ops.  Each lane writes its partial readout
+//    Σ_{own n} C h to shared memory,
 //    (3) sums the NT partials, applies D·u and the SiLU gate and writes y
 //    with 16-byte stores.  Warps synchronise only through the ring's
 //    mbarriers; every wait is bounded (kWaitBudgetCycles).
@@ -30,6 +32,7 @@
 #include <stdlib.h>
 
 #include <algorithm>
+#include <type_traits>
 
 #include "ssm_common.cuh"
 #include "ssm_internal.h"
@@ -38,6 +41,9 @@
 // Build-time tuning knobs (defaults are the measured best on B200).
 #ifndef SSM_TMA_STAGES
 #define SSM_TMA_STAGES 3      // depth of the TMA ring for bf16 io
+#endif
+#ifndef SSM_TMA_POLY_PAIRS
+#define SSM_TMA_POLY_PAIRS 0  // (state, step-pair) slots of 16 per block using ex2_poly2
 #endif
 #ifndef SSM_TMA_UNROLL
 #define SSM_TMA_UNROLL 2      // 8-step blocks unrolled in the recurrence loop
@@ -48,6 +54,7 @@ namespace ssm {
 namespace {
 
 constexpr int kTmaUnroll = SSM_TMA_UNROLL;
+constexpr int kPolyPairs = SSM_TMA_POLY_PAIRS;
 
 constexpr int align128(int x) { return (x + 127) / 128 * 128; }
 
@@ -200,6 +207,7 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
 
     float2 A2d[NS];                  // A[d, n] log2(e), duplicated for f32x2 math
     float h[NS];
+    bool poly_ok = false;            // every A of this warp <= 0 (ex2_poly2 applies)
     int bsel = 0;
     bool live = false;
     // per-item constants for the prep / epilogue rows
@@ -218,11 +226,14 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
             const int d = live ? row % p.dim : 0;
             bsel = live ? row / p.dim - q0 / p.dim : 0;
 #pragma unroll
+            bool neg = true;
             for (int j = 0; j < NS; ++j) {
                 const float a = live ? p.A[(size_t)d * N + g * NS + j] * SSM_LOG2E : 0.f;
                 A2d[j] = make_float2(a, a);
                 h[j] = 0.f;
+                neg = neg && a <= 0.f;
             }
+            poly_ok = __all_sync(0xffffffffu, neg);
 #pragma unroll
             for (int i = 0; i < IPL; ++i) {
                 const int rr = wrow0 + (lane + 32 * i) / CPR;
@@ -240,7 +251,8 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
             const T *rawD = reinterpret_cast<const T *>(st) + warp * CPW * TT;
             const T *rawU = reinterpret_cast<const T *>(st + Ly::RAW_CH) + warp * CPW * TT;
             const T *rawZ = reinterpret_cast<const T *>(st + 2 * Ly::RAW_CH) + warp * CPW * TT;
-            // (1) Δ and Δ·u, once per element
+            // (1) Δ and Δ·u, once per element (pairs of steps in f32x2 math)
+            const bool full_tile = t0 + TT <= p.L;
 #pragma unroll
             for (int i = 0; i < IPL; ++i) {
                 const int it = lane + 32 * i, rl = it / CPR, t = (it % CPR) * CHUNK;
@@ -252,11 +264,19 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                     IO<T>::unpack(*reinterpret_cast<const uint4 *>(rawD + rl * TT + t + v0), dr);
                     IO<T>::unpack(*reinterpret_cast<const uint4 *>(rawU + rl * TT + t + v0), uu);
 #pragma unroll
-                    for (int k = 0; k < V; ++k) {
-                        const float r = dr[k] + bias[i];
-                        const bool ok = irow[i] >= 0 && (t0 + t + v0 + k) < p.L;
-                        dt[v0 + k] = ok ? (p.softplus ? softplus_fast(r) : r) : 0.f;
-                        du[v0 + k] = dt[v0 + k] * uu[k];
+                    for (int k = 0; k < V; k += 2) {
+                        const float2 r = __fadd2_rn(make_float2(dr[k], dr[k + 1]), make_float2(bias[i], bias[i]));
+                        float2 d2 = p.softplus ? softplus_fast2(r) : r;
+                        if (!full_tile) {
+                            const bool ok0 = irow[i] >= 0 && (t0 + t + v0 + k) < p.L;
+                            const bool ok1 = irow[i] >= 0 && (t0 + t + v0 + k + 1) < p.L;
+                            d2 = make_float2(ok0 ? d2.x : 0.f, ok1 ? d2.y : 0.f);
+                        } else if (irow[i] < 0) {
+                            d2 = make_float2(0.f, 0.f);
+                        }
+                        const float2 u2 = __fmul2_rn(d2, make_float2(uu[k], uu[k + 1]));
+                        dt[v0 + k] = d2.x; dt[v0 + k + 1] = d2.y;
+                        du[v0 + k] = u2.x; du[v0 + k + 1] = u2.y;
                     }
                 }
 #pragma unroll
@@ -267,45 +287,60 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
             }
             __syncwarp();
             // (2) the recurrence, two time steps per f32x2 op; B and C are read
-            // in the io dtype straight from the TMA tile
+            // in the io dtype straight from the TMA tile, the eight lanes of a
+            // quarter-warp reading the same row (a broadcast load)
             const T *rawB = reinterpret_cast<const T *>(st + 3 * Ly::RAW_CH) + (bsel * N + g * NS) * TT;
             const T *rawC = reinterpret_cast<const T *>(st + 3 * Ly::RAW_CH + Ly::RAW_BC) + (bsel * N + g * NS) * TT;
             float *myY = wY + (g * CPW + c) * WS;
+            // one 8-step block of the recurrence; USE_POLY evaluates some of the
+            // exponentials with ex2_poly2 on the FMA pipe instead of the SFU
+            auto run_blocks = [&](auto use_poly) {
+                constexpr bool kPoly = decltype(use_poly)::value;
 #pragma unroll kTmaUnroll
-            for (int tb = 0; tb < TT; tb += 8) {
-                float2 dtp[4], dup[4];
-                {
-                    const float4 a = *reinterpret_cast<const float4 *>(wDt + c * WS + tb);
-                    const float4 b = *reinterpret_cast<const float4 *>(wDt + c * WS + tb + 4);
-                    const float4 e = *reinterpret_cast<const float4 *>(wDu + c * WS + tb);
-                    const float4 f = *reinterpret_cast<const float4 *>(wDu + c * WS + tb + 4);
-                    dtp[0] = make_float2(a.x, a.y); dtp[1] = make_float2(a.z, a.w);
-                    dtp[2] = make_float2(b.x, b.y); dtp[3] = make_float2(b.z, b.w);
-                    dup[0] = make_float2(e.x, e.y); dup[1] = make_float2(e.z, e.w);
-                    dup[2] = make_float2(f.x, f.y); dup[3] = make_float2(f.z, f.w);
-                }
-                float2 y2[4];
-#pragma unroll
-                for (int pp = 0; pp < 4; ++pp) y2[pp] = make_float2(0.f, 0.f);
-#pragma unroll
-                for (int j = 0; j < NS; ++j) {
-                    float2 bq[4], cq[4];
-                    load_pairs8<T>(rawB + j * TT + tb, bq);
-                    load_pairs8<T>(rawC + j * TT + tb, cq);
-#pragma unroll
-                    for (int pp = 0; pp < 4; ++pp) {
-                        const float2 arg = __fmul2_rn(dtp[pp], A2d[j]);
-                        const float a0 = ex2(arg.x), a1 = ex2(arg.y);
-                        const float2 beta = __fmul2_rn(dup[pp], bq[pp]);
-                        const float h0 = fmaf(a0, h[j], beta.x);
-                        const float h1 = fmaf(a1, h0, beta.y);
-                        h[j] = h1;
-                        y2[pp] = __ffma2_rn(cq[pp], make_float2(h0, h1), y2[pp]);
+                for (int tb = 0; tb < TT; tb += 8) {
+                    float2 dtp[4], dup[4];
+                    {
+                        const float4 a = *reinterpret_cast<const float4 *>(wDt + c * WS + tb);
+                        const float4 b = *reinterpret_cast<const float4 *>(wDt + c * WS + tb + 4);
+                        const float4 e = *reinterpret_cast<const float4 *>(wDu + c * WS + tb);
+                        const float4 f = *reinterpret_cast<const float4 *>(wDu + c * WS + tb + 4);
+                        dtp[0] = make_float2(a.x, a.y); dtp[1] = make_float2(a.z, a.w);
+                        dtp[2] = make_float2(b.x, b.y); dtp[3] = make_float2(b.z, b.w);
+                        dup[0] = make_float2(e.x, e.y); dup[1] = make_float2(e.z, e.w);
+                        dup[2] = make_float2(f.x, f.y); dup[3] = make_float2(f.z, f.w);
                     }
+                    float2 y2[4];
+#pragma unroll
+                    for (int pp = 0; pp < 4; ++pp) y2[pp] = make_float2(0.f, 0.f);
+#pragma unroll
+                    for (int j = 0; j < NS; ++j) {
+                        float2 bq[4], cq[4];
+                        load_pairs8<T>(rawB + j * TT + tb, bq);
+                        load_pairs8<T>(rawC + j * TT + tb, cq);
+#pragma unroll
+                        for (int pp = 0; pp < 4; ++pp) {
+                            const float2 arg = __fmul2_rn(dtp[pp], A2d[j]);
+                            float2 a;
+                            if (kPoly && (pp * NS + j) % 16 < kPolyPairs) {
+                                a = ex2_poly2(arg);
+                            } else {
+                                a = make_float2(ex2(arg.x), ex2(arg.y));
+                            }
+                            const float2 beta = __fmul2_rn(dup[pp], bq[pp]);
+                            const float h0 = fmaf(a.x, h[j], beta.x);
+                            const float h1 = fmaf(a.y, h0, beta.y);
+                            h[j] = h1;
+                            y2[pp] = __ffma2_rn(cq[pp], make_float2(h0, h1), y2[pp]);
+                        }
+                    }
+                    *reinterpret_cast<float4 *>(myY + tb) = make_float4(y2[0].x, y2[0].y, y2[1].x, y2[1].y);
+                    *reinterpret_cast<float4 *>(myY + tb + 4) = make_float4(y2[2].x, y2[2].y, y2[3].x, y2[3].y);
                 }
-                *reinterpret_cast<float4 *>(myY + tb) = make_float4(y2[0].x, y2[0].y, y2[1].x, y2[1].y);
-                *reinterpret_cast<float4 *>(myY + tb + 4) = make_float4(y2[2].x, y2[2].y, y2[3].x, y2[3].y);
-            }
+            };
+            if (kPolyPairs > 0 && poly_ok)
+                run_blocks(std::integral_constant<bool, true>{});
+            else
+                run_blocks(std::integral_constant<bool, false>{});
             // checkpoints and the final state
             const int tend = min(t0 + TT, p.L);
             const int row = wrow0 + c;
@@ -345,13 +380,18 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                     IO<T>::unpack(*reinterpret_cast<const uint4 *>(rawU + rl * TT + t + v0), uu);
                     if (p.has_z) IO<T>::unpack(*reinterpret_cast<const uint4 *>(rawZ + rl * TT + t + v0), zz);
 #pragma unroll
-                    for (int k = 0; k < V; ++k) {
-                        float yy = fmaf(Dd[i], uu[k], y[v0 + k]);
+                    for (int k = 0; k < V; k += 2) {
+                        float2 yy = __ffma2_rn(make_float2(Dd[i], Dd[i]), make_float2(uu[k], uu[k + 1]),
+                                               make_float2(y[v0 + k], y[v0 + k + 1]));
                         if (p.has_z) {
-                            if constexpr (sizeof(T) == 2) yy *= silu_tanh(zz[k]);
-                            else yy *= zz[k] * sigmoid(zz[k]);
+                            if constexpr (sizeof(T) == 2) {
+                                yy = __fmul2_rn(yy, silu_tanh2(make_float2(zz[k], zz[k + 1])));
+                            } else {
+                                yy.x *= zz[k] * sigmoid(zz[k]);
+                                yy.y *= zz[k + 1] * sigmoid(zz[k + 1]);
+                            }
                         }
-                        o[k] = yy;
+                        o[k] = yy.x; o[k + 1] = yy.y;
                     }
                     __stcs(reinterpret_cast<uint4 *>(out + v0), IO<T>::pack(o));
                 }
