@@ -224,6 +224,8 @@ def run_ours(args, world, rank, local):
     from selective_state_space_50_b200.workloads import WORKLOADS, generate, to_torch
 
     w = WORKLOADS[args.workload]
+    if args.seqlen:   # shorter sequence of the same workload (profiling small cases)
+        w = w.replace(seqlen=args.seqlen, name=f"{w.name}_L{args.seqlen}")
     dev = torch.device("cuda", local)
     # every rank processes its own batch of the same shape (weak scaling)
     w_rank = w.replace(seed=w.seed + 7919 * rank)
@@ -345,6 +347,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--workload", default=WORKLOAD,
                     help="workload to time (default: the Mamba-130M layer shape)")
+    ap.add_argument("--seqlen", type=int, default=0,
+                    help="override the workload's sequence length (for profiling small cases)")
     args = ap.parse_args()
     world, rank, local = dist_setup(args)
     try:

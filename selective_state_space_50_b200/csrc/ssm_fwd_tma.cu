@@ -89,7 +89,7 @@ struct TmaLayout {
     static constexpr int ITEMS = CPW * (TT / CHUNK);           // (row, chunk) items per warp
     static_assert(kTotal <= 227 * 1024, "shared memory budget");
     static_assert(TT % 8 == 0 && ITEMS % 32 == 0, "tile shape");
-    static_assert(NT == 2 || NT == 4 || NT == 8, "lane split");
+    static_assert(NT == 2 || NT == 4 || NT == 8 || NT == 16, "lane split");
 };
 
 // Loads 8 consecutive time steps of one B or C row from a raw stage tile
@@ -478,10 +478,83 @@ cudaError_t launch_cfg(const FwdParams &fp, cudaStream_t stream) {
     return cudaGetLastError();
 }
 
-// Consumer warps per CTA for each lane split and io width (as many as the
-// shared-memory budget allows), and the rows one pass of it holds.
-constexpr int nwc_for(int nt, bool bf16) { return bf16 ? (nt == 4 ? 12 : 9) : 8; }
-constexpr int rows_cap(int nt, bool bf16) { return nwc_for(nt, bf16) * (32 / nt); }
+// Launch configurations.  For a lane split NT (lanes per channel) the tile
+// holds TT = max(32, 8 * NT) steps, so every lane owns one 8-step
+// prep/epilogue item; the consumer-warp count NWC and ring depth STAGES are
+// the largest the 227 KB shared-memory budget allows (static_assert in
+// TmaLayout).
+template <typename T, int N, int NT> struct TmaCfg;
+#define SSM_TMA_CFG(T_, N_, NT_, NWC_, ST_)                                   \
+    template <> struct TmaCfg<T_, N_, NT_> {                                  \
+        static constexpr int TT = (8 * NT_ > 32 ? 8 * NT_ : 32);              \
+        static constexpr int NWC = NWC_, STAGES = ST_;                        \
+        static constexpr int MAXR = NWC_ * (32 / NT_);                        \
+    };
+using bf16_t = __nv_bfloat16;
+SSM_TMA_CFG(bf16_t, 16, 2, 9, SSM_TMA_STAGES)
+SSM_TMA_CFG(bf16_t, 16, 4, 12, SSM_TMA_STAGES)
+SSM_TMA_CFG(bf16_t, 16, 8, 12, 3)
+SSM_TMA_CFG(bf16_t, 16, 16, 7, 3)
+SSM_TMA_CFG(bf16_t, 32, 4, 12, SSM_TMA_STAGES)
+SSM_TMA_CFG(bf16_t, 32, 8, 10, 3)
+SSM_TMA_CFG(bf16_t, 32, 16, 7, 2)
+SSM_TMA_CFG(bf16_t, 8, 2, 9, SSM_TMA_STAGES)
+SSM_TMA_CFG(bf16_t, 8, 4, 12, 3)
+SSM_TMA_CFG(bf16_t, 8, 8, 12, 3)
+SSM_TMA_CFG(float, 16, 2, 8, 2)
+SSM_TMA_CFG(float, 16, 4, 8, 2)
+SSM_TMA_CFG(float, 16, 8, 8, 2)
+SSM_TMA_CFG(float, 16, 16, 6, 2)
+SSM_TMA_CFG(float, 32, 4, 8, 2)
+SSM_TMA_CFG(float, 32, 8, 6, 2)
+SSM_TMA_CFG(float, 32, 16, 3, 2)
+SSM_TMA_CFG(float, 8, 2, 8, 2)
+SSM_TMA_CFG(float, 8, 4, 8, 2)
+SSM_TMA_CFG(float, 8, 8, 8, 2)
+#undef SSM_TMA_CFG
+
+template <typename T, int N, int NT>
+cudaError_t launch_nt(const FwdParams &fp, cudaStream_t stream) {
+    using C = TmaCfg<T, N, NT>;
+    return launch_cfg<T, NT, N / NT, C::TT, C::NWC, C::STAGES>(fp, stream);
+}
+
+template <typename T, int N, int NT>
+constexpr int maxr() { return TmaCfg<T, N, NT>::MAXR; }
+
+// Lane splits available for each dstate, fewest lanes per channel first.
+template <typename T, int N>
+cudaError_t launch_n(const FwdParams &fp, int nt, cudaStream_t stream) {
+    if constexpr (N == 8) {
+        if (nt == 2) return launch_nt<T, 8, 2>(fp, stream);
+        if (nt == 4) return launch_nt<T, 8, 4>(fp, stream);
+        return launch_nt<T, 8, 8>(fp, stream);
+    } else if constexpr (N == 16) {
+        if (nt == 2) return launch_nt<T, 16, 2>(fp, stream);
+        if (nt == 4) return launch_nt<T, 16, 4>(fp, stream);
+        if (nt == 8) return launch_nt<T, 16, 8>(fp, stream);
+        return launch_nt<T, 16, 16>(fp, stream);
+    } else {
+        if (nt == 4) return launch_nt<T, 32, 4>(fp, stream);
+        if (nt == 8) return launch_nt<T, 32, 8>(fp, stream);
+        return launch_nt<T, 32, 16>(fp, stream);
+    }
+}
+
+template <typename T>
+int rows_cap(int N, int nt) {
+    if (N == 8) return nt == 2 ? maxr<T, 8, 2>() : nt == 4 ? maxr<T, 8, 4>() : maxr<T, 8, 8>();
+    if (N == 16)
+        return nt == 2 ? maxr<T, 16, 2>() : nt == 4 ? maxr<T, 16, 4>() : nt == 8 ? maxr<T, 16, 8>()
+                                                                              : maxr<T, 16, 16>();
+    return nt == 4 ? maxr<T, 32, 4>() : nt == 8 ? maxr<T, 32, 8>() : maxr<T, 32, 16>();
+}
+
+bool nt_valid(int N, int nt) {
+    if (N == 8) return nt == 2 || nt == 4 || nt == 8;
+    if (N == 16) return nt == 2 || nt == 4 || nt == 8 || nt == 16;
+    return nt == 4 || nt == 8 || nt == 16;
+}
 
 }  // namespace
 
@@ -493,30 +566,32 @@ bool try_launch_fwd_tma(const FwdParams &fp, cudaStream_t stream, cudaError_t *e
     if (!get_encode()) return false;
     const long long P = (long long)fp.batch * fp.dim;
     const int sms = sm_count();
-    if (P < 32LL * sms) return false;               // too few channels: not enough lanes
-    const long long R = (P + sms - 1) / sms;
-    // choose the lane split: 4 lanes per channel while one pass holds the rows
-    int nt = (fp.N == 8) ? 2 : (fp.N == 32 ? 4 : (R <= rows_cap(4, fp.io_bf16) ? 4 : 2));
-    // SSM_TMA_NT=2|4 overrides the lane split for dstate 16 (tuning knob)
+    if (P < sms) return false;                      // fewer channels than SMs
+    const long long R = (P + sms - 1) / sms;        // rows per SM
+    // Lane split: the fewest lanes per channel that still give every SM
+    // 8 warps of lanes (more states per lane = less per-state overhead).
+    int nt = 0;
+    for (int cand : {2, 4, 8, 16}) {
+        if (!nt_valid(fp.N, cand)) continue;
+        nt = cand;
+        if (R * cand >= 256) break;
+    }
+    // SSM_TMA_NT overrides the lane split (tuning knob)
     static const char *force_nt = getenv("SSM_TMA_NT");
-    if (fp.N == 16 && force_nt && (force_nt[0] == '2' || force_nt[0] == '4')) nt = force_nt[0] - '0';
-    const long long cap = rows_cap(nt, fp.io_bf16);
+    if (force_nt && nt_valid(fp.N, atoi(force_nt))) nt = atoi(force_nt);
+    const long long cap = fp.io_bf16 ? rows_cap<__nv_bfloat16>(fp.N, nt) : rows_cap<float>(fp.N, nt);
     const long long npass = (R + cap - 1) / cap;
     const long long rows_pass = (R + npass - 1) / npass;
     if (rows_pass > fp.dim) return false;           // a pass may touch at most two batch rows
     cudaError_t e;
     if (fp.io_bf16) {
         using T = __nv_bfloat16;
-        if (fp.N == 8) e = launch_cfg<T, 2, 4, 32, nwc_for(2, true), SSM_TMA_STAGES>(fp, stream);
-        else if (fp.N == 16) e = nt == 4 ? launch_cfg<T, 4, 4, 32, nwc_for(4, true), SSM_TMA_STAGES>(fp, stream)
-                                         : launch_cfg<T, 2, 8, 32, nwc_for(2, true), SSM_TMA_STAGES>(fp, stream);
-        else e = launch_cfg<T, 4, 8, 32, nwc_for(4, true), SSM_TMA_STAGES>(fp, stream);
+        e = fp.N == 8 ? launch_n<T, 8>(fp, nt, stream)
+          : fp.N == 16 ? launch_n<T, 16>(fp, nt, stream) : launch_n<T, 32>(fp, nt, stream);
     } else {
         using T = float;
-        if (fp.N == 8) e = launch_cfg<T, 2, 4, 32, nwc_for(2, false), 2>(fp, stream);
-        else if (fp.N == 16) e = nt == 4 ? launch_cfg<T, 4, 4, 32, nwc_for(4, false), 2>(fp, stream)
-                                         : launch_cfg<T, 2, 8, 32, nwc_for(2, false), 2>(fp, stream);
-        else e = launch_cfg<T, 4, 8, 32, nwc_for(4, false), 2>(fp, stream);
+        e = fp.N == 8 ? launch_n<T, 8>(fp, nt, stream)
+          : fp.N == 16 ? launch_n<T, 16>(fp, nt, stream) : launch_n<T, 32>(fp, nt, stream);
     }
     *err = e;
     return true;

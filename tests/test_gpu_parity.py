@@ -202,6 +202,13 @@ TMA_CASES = [
     (4, 5120, 24, 16, "bf16", True, True, True, True, "neg_lognormal"),
     (1, 4800, 1000, 16, "bf16", True, True, True, True, "neg_n1"),
     (2, 3000, 200, 16, "f32", False, False, False, True, "neg_lognormal"),
+    # fewer rows per SM: 8 and 16 lanes per channel
+    (2, 2960, 64, 16, "bf16", True, True, True, True, "neg_lognormal"),
+    (1, 2000, 264, 16, "bf16", True, True, True, True, "neg_lognormal"),
+    (1, 1500, 128, 16, "f32", True, True, True, True, "neg_lognormal"),
+    (1, 3000, 64, 32, "bf16", True, True, True, True, "neg_lognormal"),
+    (2, 2400, 64, 8, "f32", True, True, True, True, "neg_lognormal"),
+    (1, 200, 64, 16, "bf16", True, True, True, True, "neg_lognormal"),
 ]
 
 
