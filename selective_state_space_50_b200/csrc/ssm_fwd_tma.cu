@@ -77,18 +77,28 @@ struct TmaLayout {
     static constexpr int ES = sizeof(T);
     static constexpr int RAW_ROW = TT * ES;
     static constexpr int RAW_CH = align128(MAXR * RAW_ROW);
-    static constexpr int RAW_BC = align128(2 * N * RAW_ROW);   // up to two batch rows
-    static constexpr int STAGE = 3 * RAW_CH + 2 * RAW_BC;
+    // B and C tiles: when a row spans >= 128 bytes it is loaded in 128-byte
+    // pieces with the TMA 128B swizzle (16-byte chunk index XOR row % 8), so
+    // lanes reading the same chunk of different rows hit different banks.
+    static constexpr bool SWZ = RAW_ROW >= 128;
+    static constexpr int PW = SWZ ? 128 : RAW_ROW;             // bytes per piece row
+    static constexpr int NPIECE = RAW_ROW / PW;
+    static constexpr int PIECE = 2 * N * PW;                   // one piece, two batch rows
+    static constexpr int RAW_BC = NPIECE * PIECE;
+    static constexpr int kBC0 = (3 * RAW_CH + 1023) / 1024 * 1024;
+    static constexpr int STAGE = (kBC0 + 2 * RAW_BC + 1023) / 1024 * 1024;
     static constexpr int WS = TT + 4;                          // fp32 row stride (floats)
     static constexpr int WBUF = (2 + NT) * CPW * WS * 4;       // Δ, Δ·u, NT readout partials
     static constexpr int kW = STAGES * STAGE;
     static constexpr int kBar = kW + NWC * WBUF;
     static constexpr int kTotal = kBar + 2 * STAGES * 8;
+    static constexpr int kAlloc = kTotal + 1024;   // room to align the base to 1024 B
     static constexpr int kThreads = (NWC + 1) * 32;
     static constexpr int CHUNK = 8;                            // steps per prep/epilogue item
     static constexpr int ITEMS = CPW * (TT / CHUNK);           // (row, chunk) items per warp
-    static_assert(kTotal <= 227 * 1024, "shared memory budget");
+    static_assert(kAlloc <= 227 * 1024, "shared memory budget");
     static_assert(TT % 8 == 0 && ITEMS % 32 == 0, "tile shape");
+    static_assert(!SWZ || (RAW_ROW % 128 == 0 && PIECE % 1024 == 0), "swizzle atoms");
     static_assert(NT == 2 || NT == 4 || NT == 8 || NT == 16, "lane split");
 };
 
@@ -114,6 +124,25 @@ __device__ __forceinline__ void load_pairs8<float>(const float *src, float2 (&v)
     v[2] = make_float2(b.x, b.y); v[3] = make_float2(b.z, b.w);
 }
 
+// Same, for chunks at separate addresses (the swizzled layout stores the two
+// 16-byte halves of an fp32 8-step group apart; for bf16 `hi` is unused).
+template <typename T>
+__device__ __forceinline__ void load_pairs8_at(const T *lo, const T *hi, float2 (&v)[4]);
+
+template <>
+__device__ __forceinline__ void load_pairs8_at<__nv_bfloat16>(const __nv_bfloat16 *lo, const __nv_bfloat16 *,
+                                                              float2 (&v)[4]) {
+    load_pairs8<__nv_bfloat16>(lo, v);
+}
+
+template <>
+__device__ __forceinline__ void load_pairs8_at<float>(const float *lo, const float *hi, float2 (&v)[4]) {
+    const float4 a = *reinterpret_cast<const float4 *>(lo);
+    const float4 b = *reinterpret_cast<const float4 *>(hi);
+    v[0] = make_float2(a.x, a.y); v[1] = make_float2(a.z, a.w);
+    v[2] = make_float2(b.x, b.y); v[3] = make_float2(b.z, b.w);
+}
+
 template <typename T, int NT, int NS, int TT, int NWC, int STAGES>
 __global__ void __launch_bounds__((NWC + 1) * 32, 1)
 fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constant__ CUtensorMap m_u,
@@ -124,7 +153,10 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
     constexpr int IPL = Ly::ITEMS / 32;   // prep/epilogue items per lane
     constexpr int CPR = TT / CHUNK;       // chunks per row
 
-    extern __shared__ __align__(128) uint8_t smem[];
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    // 1024-byte aligned base: the 128B-swizzle pattern of the B/C tiles repeats
+    // every 1024 bytes of shared-memory address
+    uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + Ly::kBar);
     uint64_t *empty = full + STAGES;
 
@@ -181,11 +213,13 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
             tma_load_2d(st, &m_delta, t0, q0, full + s);
             tma_load_2d(st + Ly::RAW_CH, &m_u, t0, q0, full + s);
             if (p.has_z) tma_load_2d(st + 2 * Ly::RAW_CH, &m_z, t0, q0, full + s);
-            for (int bs = 0; bs < nb; ++bs) {
-                tma_load_2d(st + 3 * Ly::RAW_CH + bs * N * Ly::RAW_ROW, &m_B, t0, (b_lo + bs) * N, full + s);
-                tma_load_2d(st + 3 * Ly::RAW_CH + Ly::RAW_BC + bs * N * Ly::RAW_ROW, &m_C, t0,
-                            (b_lo + bs) * N, full + s);
-            }
+            for (int bs = 0; bs < nb; ++bs)
+                for (int pc = 0; pc < Ly::NPIECE; ++pc) {
+                    const int off = Ly::kBC0 + pc * Ly::PIECE + bs * N * Ly::PW;
+                    const int x = t0 + pc * (Ly::PW / (int)sizeof(T));
+                    tma_load_2d(st + off, &m_B, x, (b_lo + bs) * N, full + s);
+                    tma_load_2d(st + off + Ly::RAW_BC, &m_C, x, (b_lo + bs) * N, full + s);
+                }
             if (++s == STAGES) { s = 0; phase ^= 1; }
             if (++tile == ntiles) { tile = 0; ++q; }
         }
@@ -289,8 +323,18 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
             // (2) the recurrence, two time steps per f32x2 op; B and C are read
             // in the io dtype straight from the TMA tile, the eight lanes of a
             // quarter-warp reading the same row (a broadcast load)
-            const T *rawB = reinterpret_cast<const T *>(st + 3 * Ly::RAW_CH) + (bsel * N + g * NS) * TT;
-            const T *rawC = reinterpret_cast<const T *>(st + 3 * Ly::RAW_CH + Ly::RAW_BC) + (bsel * N + g * NS) * TT;
+            const uint8_t *rawB = st + Ly::kBC0;
+            const uint8_t *rawC = rawB + Ly::RAW_BC;
+            // byte address of the 16-byte chunk holding steps [tb, tb + 16/size)
+            // of state row rr (within the two-batch-row B or C tile)
+            auto bc_chunk = [&](const uint8_t *base, int rr, int tb) -> const T * {
+                const int byte = tb * (int)sizeof(T);
+                const int pc = byte / Ly::PW, in = byte % Ly::PW;
+                int chunk = in >> 4;
+                if constexpr (Ly::SWZ) chunk ^= (rr & 7);
+                return reinterpret_cast<const T *>(base + pc * Ly::PIECE + rr * Ly::PW + (chunk << 4));
+            };
+            const int rr0 = bsel * N + g * NS;
             float *myY = wY + (g * CPW + c) * WS;
             // one 8-step block of the recurrence; USE_POLY evaluates some of the
             // exponentials with ex2_poly2 on the FMA pipe instead of the SFU
@@ -315,8 +359,8 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
 #pragma unroll
                     for (int j = 0; j < NS; ++j) {
                         float2 bq[4], cq[4];
-                        load_pairs8<T>(rawB + j * TT + tb, bq);
-                        load_pairs8<T>(rawC + j * TT + tb, cq);
+                        load_pairs8_at<T>(bc_chunk(rawB, rr0 + j, tb), bc_chunk(rawB, rr0 + j, tb + 4), bq);
+                        load_pairs8_at<T>(bc_chunk(rawC, rr0 + j, tb), bc_chunk(rawC, rr0 + j, tb + 4), cq);
 #pragma unroll
                         for (int pp = 0; pp < 4; ++pp) {
                             const float2 arg = __fmul2_rn(dtp[pp], A2d[j]);
@@ -336,6 +380,7 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                     *reinterpret_cast<float4 *>(myY + tb) = make_float4(y2[0].x, y2[0].y, y2[1].x, y2[1].y);
                     *reinterpret_cast<float4 *>(myY + tb + 4) = make_float4(y2[2].x, y2[2].y, y2[3].x, y2[3].y);
                 }
+        
             };
             if (kPolyPairs > 0 && poly_ok)
                 run_blocks(std::integral_constant<bool, true>{});
@@ -420,7 +465,7 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
 }
 
 bool make_map(CUtensorMap *m, const void *base, bool bf16, uint64_t rows, uint64_t cols, uint32_t box_cols,
-              uint32_t box_rows) {
+              uint32_t box_rows, bool swizzle128 = false) {
     auto enc = get_encode();
     if (!enc) return false;
     const uint64_t es = bf16 ? 2 : 4;
@@ -430,7 +475,8 @@ bool make_map(CUtensorMap *m, const void *base, bool bf16, uint64_t rows, uint64
     cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
                      const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                     CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                     swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -457,8 +503,8 @@ cudaError_t launch_cfg(const FwdParams &fp, cudaStream_t stream) {
     if (!make_map(&md, fp.delta, bf16, P, fp.L, TT, rows_max) ||
         !make_map(&mu, fp.u, bf16, P, fp.L, TT, rows_max) ||
         !make_map(&mz, fp.z ? fp.z : fp.u, bf16, P, fp.L, TT, rows_max) ||
-        !make_map(&mB, fp.B, bf16, (uint64_t)fp.batch * fp.N, fp.L, TT, Ly::N) ||
-        !make_map(&mC, fp.C, bf16, (uint64_t)fp.batch * fp.N, fp.L, TT, Ly::N))
+        !make_map(&mB, fp.B, bf16, (uint64_t)fp.batch * fp.N, fp.L, Ly::PW / sizeof(T), Ly::N, Ly::SWZ) ||
+        !make_map(&mC, fp.C, bf16, (uint64_t)fp.batch * fp.N, fp.L, Ly::PW / sizeof(T), Ly::N, Ly::SWZ))
         return cudaErrorInvalidValue;
     TmaFwdParams p{};
     p.A = fp.A; p.D = fp.D; p.delta_bias = fp.delta_bias; p.out = fp.out;
@@ -470,11 +516,11 @@ cudaError_t launch_cfg(const FwdParams &fp, cudaStream_t stream) {
     auto kern = fwd_tma_kernel<T, NT, NS, TT, NWC, STAGES>;
     static bool attr_done = false;
     if (!attr_done) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Ly::kTotal);
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Ly::kAlloc);
         if (e != cudaSuccess) return e;
         attr_done = true;
     }
-    kern<<<grid, Ly::kThreads, Ly::kTotal, stream>>>(md, mu, mz, mB, mC, p);
+    kern<<<grid, Ly::kThreads, Ly::kAlloc, stream>>>(md, mu, mz, mB, mC, p);
     return cudaGetLastError();
 }
 
