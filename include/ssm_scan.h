@@ -153,6 +153,42 @@ ssm_status_t ssm_selective_scan_bwd(const ssm_shape_t *shape,
                                     void *stream);
 
 /*
+ * Backward selective scan that allocates nothing (the pages have no
+ * counterpart: they describe no memory management interface).
+ *
+ * For callers that cannot provide device scratch: ones with no device
+ * allocator at hand, or that must not call one (cudaMalloc and cudaFree can
+ * synchronise the whole device, and some runtimes forbid allocation after
+ * start-up), and that do not keep the forward's checkpoints.  Same arguments
+ * and results as ssm_selective_scan_bwd with ckpt = NULL, except that the
+ * checkpoint scratch comes from a static device array of
+ * SSM_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that loads
+ * the library holds until the process exits.
+ *
+ *  - Shapes whose scratch (ssm_selective_scan_bwd_scratch_bytes(shape, 0))
+ *    exceeds SSM_NOALLOC_SCRATCH_BYTES are rejected with
+ *    SSM_ERR_UNSUPPORTED before anything is launched.
+ *  - The first call on a device looks up the array's device address (once
+ *    per device, with that device current); make that first call before any
+ *    stream capture.
+ *  - Every call on a device shares the one array and overwrites it: calls
+ *    that overlap on the GPU (e.g. on two streams) race, so serialise them.
+ *    Nothing of a previous call's contents is relied upon.
+ *  - Calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+#define SSM_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+ssm_status_t ssm_selective_scan_bwd_noalloc(const ssm_shape_t *shape,
+                                            const void *u, const void *delta,
+                                            const float *A, const void *B, const void *C,
+                                            const float *D, const void *z,
+                                            const float *delta_bias, int delta_softplus,
+                                            const void *dout,
+                                            float *du, float *ddelta, float *dA,
+                                            float *dB, float *dC, float *dD, float *dz,
+                                            float *ddelta_bias, void *stream);
+
+/*
  * Synchronises `stream`, then reports (and clears) the device-side error word
  * that kernels set when one of their bounded waits gives up: SSM_OK if none
  * did since the previous call, SSM_ERR_TIMEOUT otherwise.  Kernel waits are

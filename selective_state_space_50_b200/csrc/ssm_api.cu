@@ -123,6 +123,11 @@ bool aligned16(const void *p) { return ((uintptr_t)p & 15) == 0; }
 
 }  // namespace
 
+ssm_status_t ssm::set_last_error(ssm_status_t status, const char *msg) {
+    g_last_error = msg ? msg : "";
+    return status;
+}
+
 extern "C" {
 
 int ssm_version(void) { return 100; }

@@ -45,6 +45,10 @@ cudaError_t launch_fwd(const FwdParams &p, bool states_only, cudaStream_t stream
 // Launches the TMA-fed persistent forward when it applies (returns true and
 // sets *err); returns false when the general kernel must be used.
 bool try_launch_fwd_tma(const FwdParams &p, cudaStream_t stream, cudaError_t *err);
+// Records `msg` as this thread's last error (ssm_last_error_string) and
+// returns `status`.
+ssm_status_t set_last_error(ssm_status_t status, const char *msg);
+
 // Device address of the error word that kernels set when a bounded wait
 // gives up (one word per device, looked up once per device); NULL on failure.
 int *device_error_word();

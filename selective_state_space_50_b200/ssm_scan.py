@@ -24,7 +24,9 @@ CKPT_CHUNK = 64  # SSM_CKPT_CHUNK in include/ssm_scan.h
 
 EXPORTS = ("ssm_version", "ssm_last_error_string", "ssm_selective_scan_ckpt_bytes",
            "ssm_selective_scan_fwd", "ssm_selective_scan_bwd_scratch_bytes",
-           "ssm_selective_scan_bwd", "ssm_device_error_status")
+           "ssm_selective_scan_bwd", "ssm_device_error_status",
+           "ssm_selective_scan_bwd_noalloc")
+NOALLOC_SCRATCH_BYTES = 32 << 20  # SSM_NOALLOC_SCRATCH_BYTES in include/ssm_scan.h
 
 
 class SSMError(RuntimeError):
@@ -64,6 +66,8 @@ def load_library(path: str = LIB_PATH):
     lib.ssm_selective_scan_bwd.restype = i
     lib.ssm_device_error_status.argtypes = [vp]
     lib.ssm_device_error_status.restype = i
+    lib.ssm_selective_scan_bwd_noalloc.argtypes = [sp] + [vp] * 8 + [i] + [vp] * 10
+    lib.ssm_selective_scan_bwd_noalloc.restype = i
     _lib = lib
     return lib
 
@@ -134,6 +138,17 @@ def bwd_raw(shape: Shape, u, delta, A, B, C, D, z, delta_bias, delta_softplus: b
         _ptr(delta_bias), int(bool(delta_softplus)), _ptr(dout), _ptr(ckpt), _ptr(du),
         _ptr(ddelta), _ptr(dA), _ptr(dB), _ptr(dC), _ptr(dD), _ptr(dz), _ptr(ddelta_bias),
         _ptr(scratch), ctypes.c_size_t(nbytes), _stream_ptr(stream)))
+
+
+def bwd_noalloc_raw(shape: Shape, u, delta, A, B, C, D, z, delta_bias, delta_softplus: bool,
+                    dout, du, ddelta, dA, dB, dC, dD, dz, ddelta_bias, stream=None):
+    """Direct call of ssm_selective_scan_bwd_noalloc: the backward for callers
+    that can neither allocate device memory nor pass scratch; its checkpoint
+    scratch is a static array inside the library (see include/ssm_scan.h)."""
+    _check(load_library().ssm_selective_scan_bwd_noalloc(
+        ctypes.byref(shape), _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+        _ptr(delta_bias), int(bool(delta_softplus)), _ptr(dout), _ptr(du), _ptr(ddelta), _ptr(dA),
+        _ptr(dB), _ptr(dC), _ptr(dD), _ptr(dz), _ptr(ddelta_bias), _stream_ptr(stream)))
 
 
 def _need(t, name, dtype=None, cuda=True):
