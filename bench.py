@@ -48,13 +48,23 @@ def measured_peaks():
     return {"hbm_gbs": FALLBACK_HBM_GBS, "sm_max_mhz": 1965.0}, "fallback"
 
 
-def algorithmic_bytes(w, io_bytes, with_last_state=True):
+def algorithmic_bytes(w, io_bytes, with_last_state=True, backward=False):
+    """HBM bytes a fused forward must move (and, with backward, the backward
+    too): every input read once, every output written once."""
     e = w.batch * w.dim * w.seqlen
+    bc = w.batch * w.dstate * w.seqlen
     n = e * io_bytes * (3 + 1)                          # u, delta, z in; out
-    n += 2 * w.batch * w.dstate * w.seqlen * io_bytes   # B, C
+    n += 2 * bc * io_bytes                              # B, C
     n += w.dim * w.dstate * 4 + 2 * w.dim * 4           # A, D, bias
     if with_last_state:
         n += w.batch * w.dim * w.dstate * 4
+    if backward:
+        nck = -(-w.seqlen // 64)
+        ck = w.batch * w.dim * nck * w.dstate * 4
+        n += ck                                         # forward writes checkpoints
+        n += e * io_bytes * 4 + 2 * bc * io_bytes + ck  # u, delta, z, dout, B, C, ckpt read
+        n += e * 4 * 3 + 2 * bc * 4                     # du, ddelta, dz, dB, dC written
+        n += w.dim * w.dstate * 4 + 2 * w.dim * 4       # dA, dD, dbias
     return n
 
 
@@ -229,17 +239,38 @@ def run_ours(args, world, rank, local):
     dev = torch.device("cuda", local)
     # every rank processes its own batch of the same shape (weak scaling)
     w_rank = w.replace(seed=w.seed + 7919 * rank)
-    inp = generate(w_rank)
+    fwdbwd = w.name.startswith("mamba130m_layer_fwdbwd")
+    inp = generate(w_rank, with_dout=fwdbwd)
     dv = to_torch(inp, w_rank, dev)
     shape = ssm_scan.make_shape(w.batch, w.dim, w.seqlen, w.dstate, dv["u"].dtype)
     out = torch.empty_like(dv["u"])
     last = torch.empty(w.batch, w.dim, w.dstate, device=dev, dtype=torch.float32)
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    if fwdbwd:
+        ck = torch.empty(ssm_scan.ckpt_numel(shape), device=dev, dtype=torch.float32)
+        f32 = dict(device=dev, dtype=torch.float32)
+        grads = {k: torch.empty(dv[src].shape, **f32) for k, src in
+                 (("du", "u"), ("ddelta", "u"), ("dz", "u"), ("dA", "A"), ("dB", "B"), ("dC", "C"),
+                  ("dD", "D"), ("ddelta_bias", "delta_bias"))}
+        bwd_only = os.environ.get("SSM_BENCH_BWD_ONLY") == "1"
 
-    def fwd():
-        ssm_scan.fwd_raw(shape, dv["u"], dv["delta"], dv["A"], dv["B"], dv["C"], dv["D"], dv["z"],
-                         dv["delta_bias"], True, out, last, None, stream)
+        def fwd():
+            # one training step of the scan: forward keeping checkpoints, backward
+            if not bwd_only:
+                ssm_scan.fwd_raw(shape, dv["u"], dv["delta"], dv["A"], dv["B"], dv["C"], dv["D"],
+                                 dv["z"], dv["delta_bias"], True, out, last, ck, stream)
+            ssm_scan.bwd_raw(shape, dv["u"], dv["delta"], dv["A"], dv["B"], dv["C"], dv["D"],
+                             dv["z"], dv["delta_bias"], True, dv["dout"], ck, grads["du"],
+                             grads["ddelta"], grads["dA"], grads["dB"], grads["dC"], grads["dD"],
+                             grads["dz"], grads["ddelta_bias"], None, stream)
+        if bwd_only:   # checkpoints for the timed backward-only steps
+            ssm_scan.fwd_raw(shape, dv["u"], dv["delta"], dv["A"], dv["B"], dv["C"], dv["D"],
+                             dv["z"], dv["delta_bias"], True, out, last, ck, stream)
+    else:
+        def fwd():
+            ssm_scan.fwd_raw(shape, dv["u"], dv["delta"], dv["A"], dv["B"], dv["C"], dv["D"],
+                             dv["z"], dv["delta_bias"], True, out, last, None, stream)
 
     for _ in range(max(3, args.warmup)):
         flush.zero_()
@@ -266,10 +297,11 @@ def run_ours(args, world, rank, local):
     # ---- end to end through the binding, host buffers, copies inside the step
     e2e_steps = max(5, min(args.steps, 50))
     host = {k: dv[k].cpu().pin_memory() for k in ("u", "delta", "z", "B", "C", "A", "D",
-                                                   "delta_bias")}
+                                                   "delta_bias") + (("dout",) if fwdbwd else ())}
     out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    du_h = torch.empty(out.shape, dtype=torch.float32).pin_memory() if fwdbwd else None
     h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = out_h.numel() * out_h.element_size()
+    d2h = out_h.numel() * out_h.element_size() + (du_h.numel() * 4 if fwdbwd else 0)
     e_s = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
     e_e = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
     dtmp = {k: torch.empty_like(v) for k, v in dv.items() if v is not None}
@@ -277,9 +309,15 @@ def run_ours(args, world, rank, local):
     def e2e_step():
         for k, t in host.items():
             dtmp[k].copy_(t, non_blocking=True)
-        o, _, _ = ssm_scan.selective_scan_fwd(dtmp["u"], dtmp["delta"], dtmp["A"], dtmp["B"],
-                                              dtmp["C"], dtmp["D"], dtmp["z"], dtmp["delta_bias"],
-                                              True, return_last_state=True, out=out)
+        o, _, ckp = ssm_scan.selective_scan_fwd(dtmp["u"], dtmp["delta"], dtmp["A"], dtmp["B"],
+                                                dtmp["C"], dtmp["D"], dtmp["z"], dtmp["delta_bias"],
+                                                True, return_last_state=True, out=out,
+                                                return_ckpt=fwdbwd)
+        if fwdbwd:
+            g = ssm_scan.selective_scan_bwd(dtmp["u"], dtmp["delta"], dtmp["A"], dtmp["B"],
+                                            dtmp["C"], dtmp["D"], dtmp["z"], dtmp["delta_bias"],
+                                            True, dtmp["dout"], ckpt=ckp)
+            du_h.copy_(g["du"], non_blocking=True)
         out_h.copy_(o, non_blocking=True)
     for _ in range(3):
         e2e_step()
@@ -298,16 +336,21 @@ def run_ours(args, world, rank, local):
         return
     peaks, peak_src = measured_peaks()
     mean_s = t_dev / args.steps
-    ex2 = w.batch * w.dim * w.seqlen * w.dstate
+    # one exponential per (step, state) in the forward, and one more in the
+    # backward (its minimum with checkpoints)
+    ex2 = w.batch * w.dim * w.seqlen * w.dstate * (2 if fwdbwd else 1)
     sm_max = float(peaks.get("sm_max_mhz") or 1965.0)
     mufu_peak = SM_COUNT_B200 * MUFU_EX2_PER_CLK_PER_SM * sm_max * 1e6
     achieved = ex2 / mean_s
-    alg_bytes = algorithmic_bytes(w, 2 if w.io_dtype == "bf16" else 4)
+    alg_bytes = algorithmic_bytes(w, 2 if w.io_dtype == "bf16" else 4, backward=fwdbwd)
     traffic = None
-    tp = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(tp):
+    tp = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if os.path.exists(tp) and not fwdbwd:
         with open(tp) as f:
-            traffic = json.load(f).get("ssm_fwd_" + w.name)
+            for line in f:
+                parts = line.split()
+                if len(parts) == 2 and not line.startswith("#") and parts[0] == "ssm_fwd_" + w.name:
+                    traffic = int(parts[1])
     line = {
         "metric": METRIC, "value": elems_all / t_max, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": max(3, args.warmup),
@@ -328,7 +371,7 @@ def run_ours(args, world, rank, local):
         "clocks": clk.summary(),
         "e2e": {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps * (2 if fwdbwd else 1),
     }
     if world == 1 and not args.no_cpu_baseline:
         rate, cores, desc = cpu_oracle_rate(w, inp, args.cpu_budget)
