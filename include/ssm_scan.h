@@ -77,8 +77,9 @@ typedef struct {
     ssm_dtype_t io_dtype; /* dtype of u, delta, z, B, C, out, dout */
 } ssm_shape_t;
 
-/* Steps between two saved states in the forward's checkpoint buffer. */
-#define SSM_CKPT_CHUNK 64
+/* Steps between two saved states in the forward's checkpoint buffer.  The
+ * backward recomputes each such window of steps once from its saved state. */
+#define SSM_CKPT_CHUNK 8
 
 /* Library version, major * 10000 + minor * 100 + patch. */
 int ssm_version(void);

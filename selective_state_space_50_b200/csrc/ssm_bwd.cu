@@ -327,8 +327,8 @@ static cudaError_t launch_bwd_cfg(const BwdParams &p, cudaStream_t stream) {
 template <typename T>
 static cudaError_t launch_bwd_t(const BwdParams &p, cudaStream_t stream) {
     switch (p.N) {
-    case 1: return launch_bwd_cfg<T, 1, 1, 64, 32>(p, stream);
-    case 2: return launch_bwd_cfg<T, 1, 2, 64, 16>(p, stream);
+    case 1: return launch_bwd_cfg<T, 1, 1, 64, 8>(p, stream);
+    case 2: return launch_bwd_cfg<T, 1, 2, 64, 8>(p, stream);
     case 4: return launch_bwd_cfg<T, 1, 4, 64, 8>(p, stream);
     case 8: return launch_bwd_cfg<T, 2, 4, 32, 8>(p, stream);
     case 16: return launch_bwd_cfg<T, 4, 4, 32, 8>(p, stream);
@@ -338,6 +338,8 @@ static cudaError_t launch_bwd_t(const BwdParams &p, cudaStream_t stream) {
 }
 
 cudaError_t launch_bwd(const BwdParams &p, cudaStream_t stream) {
+    cudaError_t err = cudaSuccess;
+    if (try_launch_bwd_tma(p, stream, &err)) return err;
     return p.io_bf16 ? launch_bwd_t<__nv_bfloat16>(p, stream) : launch_bwd_t<float>(p, stream);
 }
 

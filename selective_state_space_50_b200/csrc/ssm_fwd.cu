@@ -76,7 +76,7 @@ fwd_kernel(const FwdParams p) {
     constexpr int V = IO<T>::kVec;
     constexpr int VPR = TT / V;
     static_assert(TT % V == 0 && TT % 4 == 0, "tile must hold whole vectors");
-    static_assert(SSM_CKPT_CHUNK % TT == 0, "tiles must not straddle checkpoints");
+    static_assert(TT % SSM_CKPT_CHUNK == 0 && SSM_CKPT_CHUNK % 4 == 0, "checkpoint grid");
 
     extern __shared__ __align__(16) float smem[];
     float *sDt = smem + S::kDt, *sDu = smem + S::kDu, *sU = smem + S::kU, *sZ = smem + S::kZ;
@@ -199,16 +199,17 @@ fwd_kernel(const FwdParams p) {
             }
             if (MODE == 0)
                 *reinterpret_cast<float4 *>(sY + (g * G + c) * RS + t) = make_float4(yv[0], yv[1], yv[2], yv[3]);
+            // checkpoint: state at the end of chunk k (steps past L leave it unchanged)
+            if (p.ckpt && live && (t + 4) % SSM_CKPT_CHUNK == 0) {
+                const int k = (t0 + t + 4) / SSM_CKPT_CHUNK - 1;
+                if (k * SSM_CKPT_CHUNK < L) {
+                    float *dst = p.ckpt + (((row_bd0 + d) * p.n_ckpt + k) * N + g * NS);
+#pragma unroll
+                    for (int s = 0; s < NS; ++s) dst[s] = h[s];
+                }
+            }
         }
 
-        // checkpoint: state after the last valid step of a finished chunk
-        const int tend = t0 + nvalid;
-        if (p.ckpt && live && (tend % SSM_CKPT_CHUNK == 0 || tend == L)) {
-            const int k = (tend - 1) / SSM_CKPT_CHUNK;
-            float *dst = p.ckpt + (((row_bd0 + d) * p.n_ckpt + k) * N + g * NS);
-#pragma unroll
-            for (int s = 0; s < NS; ++s) dst[s] = h[s];
-        }
         __syncthreads();
 
         // ---------------- (3) epilogue: Σ partials, D skip, gate, store

@@ -278,7 +278,8 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                 bias[i] = (ok && p.delta_bias) ? p.delta_bias[dd] : 0.f;
             }
         }
-        if (!mbar_wait(full + s, phase, p.err)) return;
+        // every lane waits; the warp leaves together if any wait gave up
+        if (!__all_sync(0xffffffffu, mbar_wait(full + s, phase, p.err))) return;
 
         if (wrow0 < q1) {
             const uint8_t *st = smem + s * Ly::STAGE;
@@ -336,6 +337,8 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
             };
             const int rr0 = bsel * N + g * NS;
             float *myY = wY + (g * CPW + c) * WS;
+            float *ck_row = (live && p.ckpt) ? p.ckpt + (size_t)(wrow0 + c) * p.n_ckpt * N + g * NS : nullptr;
+            static_assert(SSM_CKPT_CHUNK == 8, "checkpoints are written per 8-step block");
             // one 8-step block of the recurrence; USE_POLY evaluates some of the
             // exponentials with ex2_poly2 on the FMA pipe instead of the SFU
             auto run_blocks = [&](auto use_poly) {
@@ -379,6 +382,12 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                     }
                     *reinterpret_cast<float4 *>(myY + tb) = make_float4(y2[0].x, y2[0].y, y2[1].x, y2[1].y);
                     *reinterpret_cast<float4 *>(myY + tb + 4) = make_float4(y2[2].x, y2[2].y, y2[3].x, y2[3].y);
+                    // checkpoint: the state after this 8-step block (a chunk)
+                    if (ck_row && t0 + tb < p.L) {
+                        float *dst = ck_row + (size_t)((t0 + tb) / SSM_CKPT_CHUNK) * N;
+#pragma unroll
+                        for (int j = 0; j < NS; ++j) dst[j] = h[j];
+                    }
                 }
         
             };
@@ -386,14 +395,8 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                 run_blocks(std::integral_constant<bool, true>{});
             else
                 run_blocks(std::integral_constant<bool, false>{});
-            // checkpoints and the final state
-            const int tend = min(t0 + TT, p.L);
+            // the final state
             const int row = wrow0 + c;
-            if (live && p.ckpt && (tend % SSM_CKPT_CHUNK == 0 || tend == p.L)) {
-                float *dst = p.ckpt + ((size_t)row * p.n_ckpt + (tend - 1) / SSM_CKPT_CHUNK) * N + g * NS;
-#pragma unroll
-                for (int j = 0; j < NS; ++j) dst[j] = h[j];
-            }
             if (live && p.last_state && tile == ntiles - 1) {
                 float *dst = p.last_state + (size_t)row * N + g * NS;
 #pragma unroll

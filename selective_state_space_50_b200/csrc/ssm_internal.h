@@ -56,5 +56,10 @@ int *device_error_word();
 // clears it when set.
 cudaError_t read_and_clear_device_error(int *value, cudaStream_t stream);
 cudaError_t launch_bwd(const BwdParams &p, cudaStream_t stream);
+// Launches the TMA-fed persistent backward when it applies (dstate 16, 16-byte
+// aligned rows and checkpoints, at least one channel row per SM); returns
+// false when the general backward must be used.  SSM_BWD_KERNEL=general in
+// the environment disables it.
+bool try_launch_bwd_tma(const BwdParams &p, cudaStream_t stream, cudaError_t *err);
 
 }  // namespace ssm

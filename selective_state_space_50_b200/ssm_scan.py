@@ -20,7 +20,7 @@ LIB_PATH = os.environ.get("SSM_LIB_PATH") or os.path.join(_HERE, "libssmscan.so"
 
 SSM_OK, SSM_ERR_INVALID_ARG, SSM_ERR_UNSUPPORTED, SSM_ERR_CUDA, SSM_ERR_TIMEOUT = range(5)
 SSM_F32, SSM_BF16 = 0, 1
-CKPT_CHUNK = 64  # SSM_CKPT_CHUNK in include/ssm_scan.h
+CKPT_CHUNK = 8  # SSM_CKPT_CHUNK in include/ssm_scan.h
 
 EXPORTS = ("ssm_version", "ssm_last_error_string", "ssm_selective_scan_ckpt_bytes",
            "ssm_selective_scan_fwd", "ssm_selective_scan_bwd_scratch_bytes",

@@ -188,6 +188,30 @@ def test_bwd_layer_shape_full():
     check_bwd(WORKLOADS["mamba130m_layer_fwdbwd"], use_ckpt=True)
 
 
+# Shapes with dstate 16, 16-byte aligned rows and at least one channel row per
+# SM take the TMA-fed persistent backward; these cover its ragged last tile and
+# window, fp32 io, several passes per CTA, CTAs whose rows span two batch rows,
+# CTAs with mostly idle warps, and the optional inputs switched off.
+BWD_TMA_CASES = [
+    # batch, dim, L, N, io, z, D, bias, softplus, A_dist
+    (2, 2400, 72, 16, "bf16", True, True, True, True, "neg_lognormal"),
+    (3, 2000, 40, 16, "f32", True, False, True, True, "neg_lognormal"),
+    (2, 15000, 16, 16, "bf16", True, True, True, True, "neg_lognormal"),
+    (1, 4800, 1000, 16, "bf16", True, True, True, True, "neg_n1"),
+    (2, 3000, 200, 16, "f32", False, False, False, True, "neg_lognormal"),
+    (2, 2400, 64, 16, "bf16", True, True, True, False, "neg_lognormal"),
+    (1, 200, 64, 16, "bf16", True, True, True, True, "neg_lognormal"),
+    (1, 1500, 132, 16, "f32", True, True, True, True, "neg_lognormal"),
+    (4, 700, 256, 16, "bf16", False, True, True, True, "neg_lognormal"),
+]
+
+
+@pytest.mark.parametrize("case", BWD_TMA_CASES)
+@pytest.mark.parametrize("use_ckpt", [True, False])
+def test_bwd_tma_path(case, use_ckpt):
+    check_bwd(small_workload(*case), use_ckpt)
+
+
 # ------------------------------------------------------------------ TMA forward path
 # Shapes with >= 32 channels per SM and L a multiple of 8 take the TMA-fed
 # persistent kernel; these cover its ragged last tile, fp32 io, N = 8 / 32,
@@ -262,6 +286,35 @@ def _run_forced(kernel, shape_args):
                        timeout=600)
     assert r.returncode == 0, r.stderr[-2000:]
     return r.stdout
+
+
+def test_forced_general_backward():
+    """SSM_BWD_KERNEL=general keeps a shape the TMA backward covers on the
+    general kernel; both agree with the oracle."""
+    import os
+    import subprocess
+    import sys
+    code = (
+        "import sys; sys.path.insert(0, %r); sys.path.insert(0, %r)\n"
+        "import torch, numpy as np, oracle\n"
+        "from selective_state_space_50_b200 import ssm_scan\n"
+        "from selective_state_space_50_b200.workloads import Workload, generate, to_torch\n"
+        "w = Workload('f', 2, 64, 1200, 16, 'bf16', seed=6, A_dist='neg_lognormal', D_dist='u0.5_1.5')\n"
+        "inp = generate(w, with_dout=True); dv = to_torch(inp, w, 'cuda')\n"
+        "g = ssm_scan.selective_scan_bwd(dv['u'], dv['delta'], dv['A'], dv['B'], dv['C'], dv['D'],"
+        " dv['z'], dv['delta_bias'], True, dv['dout'])\n"
+        "torch.cuda.synchronize()\n"
+        "ref = oracle.bwd_workload(inp, w)\n"
+        "print('maxrel', max(float(np.linalg.norm(g[k].double().cpu().numpy() - ref[k]) /"
+        " np.linalg.norm(ref[k])) for k in ref))\n"
+    ) % (os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+         os.path.dirname(os.path.abspath(__file__)))
+    for kern in ("general", "auto"):
+        env = dict(os.environ, SSM_BWD_KERNEL=kern)
+        r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True,
+                           timeout=600)
+        assert r.returncode == 0, r.stderr[-2000:]
+        assert float(r.stdout.split()[-1]) <= 1e-3, r.stdout
 
 
 def test_forced_kernel_selection():

@@ -68,7 +68,7 @@ def test_noalloc_matches_regular_backward_on_two_calls(io):
 
 def test_noalloc_rejects_shapes_beyond_its_buffer():
     lib = ssm_scan.load_library()
-    # 8 x 1536 channels x 8192 steps needs 8*1536*128*16*4 B = 96 MiB of checkpoints
+    # 8 x 1536 channels x 8192 steps needs 8*1536*1024*16*4 B = 768 MiB of checkpoints
     shape = ssm_scan.make_shape(8, 1536, 8192, 16, torch.bfloat16)
     assert ssm_scan.bwd_scratch_bytes(shape, False) > ssm_scan.NOALLOC_SCRATCH_BYTES
     st = lib.ssm_selective_scan_bwd_noalloc(ctypes.byref(shape), *([None] * 8), 1,
