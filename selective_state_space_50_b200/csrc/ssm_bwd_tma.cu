@@ -43,6 +43,12 @@ namespace ssm {
 
 namespace {
 
+// Unroll factor of the loop over the 8-step windows of a tile.
+#ifndef SSM_BWD_WIN_UNROLL
+#define SSM_BWD_WIN_UNROLL 1
+#endif
+constexpr int kWinUnroll = SSM_BWD_WIN_UNROLL;
+
 constexpr int bwd_align128(int x) { return (x + 127) / 128 * 128; }
 constexpr int bwd_align1024(int x) { return (x + 1023) / 1024 * 1024; }
 
@@ -69,6 +75,9 @@ struct BwdLayout {
     static constexpr int RAW_BC = NPIECE * PIECE;
     static constexpr int kBC0 = bwd_align1024(4 * RAW_CH);
     static constexpr int STAGE = bwd_align1024(kBC0 + 2 * RAW_BC);
+    // B and C of a tile in fp32, [B or C][batch row][state][TT] with swizzled
+    // 16-byte chunks; two buffers (tiles alternate)
+    static constexpr int BCF = 2 * 2 * N * TT;                         // floats per buffer
     static constexpr int W = 8;                                        // window = checkpoint chunk
     static constexpr int NWIN = TT / W;
     static constexpr int WS = TT + 4;                                  // row of wDt / wDu / wGy
@@ -78,25 +87,29 @@ struct BwdLayout {
     static constexpr int kWp = 3 * CPW * WS;                           // [3][NT][CPW][PS]
     static constexpr int kWx = kWp + 3 * NT * CPW * PS;                // [32][XS]
     static constexpr int WBUF = (kWx + 32 * XS) * 4;
-    // dB/dC tile accumulator: [B or C][batch row][state, permuted][DS]
-    static constexpr int DS = TT + 8;
-    static constexpr int DBC_PAR = 2 * 2 * N * DS;
-    static constexpr int kW = STAGES * STAGE;
+    // dB/dC tile accumulator: [B or C][batch row][state][TT], rows rotated
+    static constexpr int DBC_PAR = 2 * 2 * N * TT;
+    static constexpr int kBCF = STAGES * STAGE;
+    static constexpr int kW = kBCF + 2 * BCF * 4;
     static constexpr int kDBC = kW + NWC * WBUF;
     static constexpr int kBar = kDBC + 2 * DBC_PAR * 4;
-    static constexpr int kTotal = kBar + (2 * STAGES + 4) * 8;
+    static constexpr int kTotal = kBar + (2 * STAGES + 6) * 8;
     static constexpr int kAlloc = kTotal + 1024;
     static constexpr int kThreads = (NWC + 1) * 32;
     static_assert(kAlloc <= 227 * 1024, "shared memory budget");
     static_assert(CPW * (TT / W) == 32, "one prep item of 8 steps per lane");
     static_assert(SSM_CKPT_CHUNK == W, "windows are checkpoint chunks");
-    static_assert(PS % 4 == 0 && XS % 4 == 0 && WS % 4 == 0 && DS % 4 == 0, "16-byte rows");
+    static_assert(PS % 4 == 0 && WS % 4 == 0 && XS == 36 && TT == 32, "row shapes");
 };
 
-// Row of state n in the dB/dC accumulator.  Lanes of different quarter-warps
-// add to different states at once; with this order and a row of DS = 40
-// floats they fall in different banks.
-__device__ __forceinline__ int dbc_row(int n) { return (n % 4) * 4 + n / 4; }
+// Column of step t of state n in the dB/dC accumulator.  The rotation puts
+// the 32 (state, step) cells that one atomic instruction of a warp touches
+// into 32 different banks.
+__device__ __forceinline__ int dbc_col(int n, int t) { return (t + 8 * (n >> 2) + (n & 3)) & 31; }
+
+// Physical 16-byte chunk of chunk `ch` in row `row` of the fp32 B/C tile:
+// the four state groups of a warp read different banks.
+__device__ __forceinline__ int bcf_chunk(int row, int ch) { return ch ^ ((row >> 2) & 7); }
 
 __device__ __forceinline__ void red_add_v4(float *addr, float4 v) {
     asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(v.x), "f"(v.y),
@@ -104,31 +117,15 @@ __device__ __forceinline__ void red_add_v4(float *addr, float4 v) {
                  : "memory");
 }
 
-// The 8 steps of one window of one row of B or C, kept packed in registers.
-template <typename T> struct BCWin;
-
-// at() unpacks with opaque instructions so that the compiler re-extracts a
-// value where it is used instead of keeping all unpacked values alive across
-// the recompute and the reverse sweep.
-template <> struct BCWin<__nv_bfloat16> {
-    uint4 v;
-    __device__ __forceinline__ float at(int t) const {
-        const uint32_t x = (t < 2) ? v.x : (t < 4) ? v.y : (t < 6) ? v.z : v.w;
-        uint32_t r;
-        if (t & 1) asm volatile("and.b32 %0, %1, 0xffff0000;" : "=r"(r) : "r"(x));
-        else asm volatile("shl.b32 %0, %1, 16;" : "=r"(r) : "r"(x));
-        return __uint_as_float(r);
-    }
-};
-
-template <> struct BCWin<float> {
-    uint4 v[2];
-    __device__ __forceinline__ float at(int t) const {
-        const uint4 &q = v[t / 4];
-        const int i = t % 4;
-        return __uint_as_float(i == 0 ? q.x : i == 1 ? q.y : i == 2 ? q.z : q.w);
-    }
-};
+// Read-only 16-byte load issued where it stands in the program, so that a
+// prefetch is not moved next to its use.
+__device__ __forceinline__ float4 ldg_f4_now(const float *ptr) {
+    float4 v;
+    asm volatile("ld.global.nc.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "l"(ptr));
+    return v;
+}
 
 __device__ __forceinline__ float4 f4add(float4 a, float4 b) {
     const float2 lo = __fadd2_rn(make_float2(a.x, a.y), make_float2(b.x, b.y));
@@ -136,7 +133,7 @@ __device__ __forceinline__ float4 f4add(float4 a, float4 b) {
     return make_float4(lo.x, lo.y, hi.x, hi.y);
 }
 
-template <typename T, int NWC, int STAGES>
+template <typename T, int NWC, int STAGES, bool HZ, bool SP>
 __global__ void __launch_bounds__((NWC + 1) * 32, 1)
 bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constant__ CUtensorMap m_u,
                const __grid_constant__ CUtensorMap m_z, const __grid_constant__ CUtensorMap m_g,
@@ -144,7 +141,7 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                const TmaBwdParams p) {
     using Ly = BwdLayout<T, NWC, STAGES>;
     constexpr int N = Ly::N, NT = Ly::NT, NS = Ly::NS, TT = Ly::TT, CPW = Ly::CPW;
-    constexpr int WS = Ly::WS, PS = Ly::PS, XS = Ly::XS, DS = Ly::DS, W = Ly::W;
+    constexpr int WS = Ly::WS, PS = Ly::PS, XS = Ly::XS, W = Ly::W;
 
     extern __shared__ __align__(128) uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -152,7 +149,9 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
     uint64_t *empty = full + STAGES;
     uint64_t *dfull = empty + STAGES;   // all consumers added their dB/dC of a tile
     uint64_t *dempty = dfull + 2;       // the producer flushed and cleared that buffer
+    uint64_t *bcready = dempty + 2;     // the producer converted B/C of a tile to fp32
     float *dbc = reinterpret_cast<float *>(smem + Ly::kDBC);
+    float *bcf = reinterpret_cast<float *>(smem + Ly::kBCF);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int G = gridDim.x;
@@ -171,6 +170,7 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
         for (int b = 0; b < 2; ++b) {
             mbar_init(dfull + b, NWC);
             mbar_init(dempty + b, 1);
+            mbar_init(bcready + b, 1);
         }
         fence_barrier_init();
     }
@@ -181,84 +181,127 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
         q0 = r0 + (int)((long long)q * R / npass);
         q1 = r0 + (int)((long long)(q + 1) * R / npass);
     };
+    // batch rows [b_lo, b_lo + nb) touched by pass q
+    auto pass_batches = [&](int q, int &b_lo, int &nb) {
+        int q0, q1;
+        pass_rows(q, q0, q1);
+        b_lo = q0 / p.dim;
+        nb = (q1 - 1) / p.dim - b_lo + 1;
+    };
 
     if (warp == NWC) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             prefetch_tensormap(&m_delta);
             prefetch_tensormap(&m_u);
-            if (p.has_z) prefetch_tensormap(&m_z);
+            if constexpr (HZ) prefetch_tensormap(&m_z);
             prefetch_tensormap(&m_g);
             prefetch_tensormap(&m_B);
             prefetch_tensormap(&m_C);
         }
-        int is_ = 0, is_s = 0, is_q = 0, is_k = 0, is_q0 = 0, is_q1 = 0;
-        auto issue_next = [&]() {   // lane 0 only
-            if (is_k == 0) pass_rows(is_q, is_q0, is_q1);
-            const int t0 = (ntiles - 1 - is_k) * TT;
-            const int b_lo = is_q0 / p.dim, nb = (is_q1 - 1) / p.dim - b_lo + 1;
-            uint8_t *st = smem + is_s * Ly::STAGE;
-            const uint32_t bytes = (uint32_t)(p.rows_max * Ly::RAW_ROW * (3 + p.has_z) +
+        int is_ = 0;
+        auto issue = [&](int kk) {   // lane 0: TMA loads of tile kk into stage kk % STAGES
+            const int q = kk / ntiles, k = kk - q * ntiles, st_i = kk % STAGES;
+            int q0, q1, b_lo, nb;
+            pass_rows(q, q0, q1);
+            pass_batches(q, b_lo, nb);
+            const int t0 = (ntiles - 1 - k) * TT;
+            uint8_t *st = smem + st_i * Ly::STAGE;
+            const uint32_t bytes = (uint32_t)(p.rows_max * Ly::RAW_ROW * (3 + (HZ ? 1 : 0)) +
                                               2 * nb * N * Ly::RAW_ROW);
-            mbar_arrive_expect_tx(full + is_s, bytes);
-            tma_load_2d(st, &m_delta, t0, is_q0, full + is_s);
-            tma_load_2d(st + Ly::RAW_CH, &m_u, t0, is_q0, full + is_s);
-            if (p.has_z) tma_load_2d(st + 2 * Ly::RAW_CH, &m_z, t0, is_q0, full + is_s);
-            tma_load_2d(st + 3 * Ly::RAW_CH, &m_g, t0, is_q0, full + is_s);
+            mbar_arrive_expect_tx(full + st_i, bytes);
+            tma_load_2d(st, &m_delta, t0, q0, full + st_i);
+            tma_load_2d(st + Ly::RAW_CH, &m_u, t0, q0, full + st_i);
+            if constexpr (HZ) tma_load_2d(st + 2 * Ly::RAW_CH, &m_z, t0, q0, full + st_i);
+            tma_load_2d(st + 3 * Ly::RAW_CH, &m_g, t0, q0, full + st_i);
             for (int bs = 0; bs < nb; ++bs)
                 for (int pc = 0; pc < Ly::NPIECE; ++pc) {
                     const int off = Ly::kBC0 + pc * Ly::PIECE + bs * N * Ly::PW;
                     const int x = t0 + pc * (Ly::PW / (int)sizeof(T));
-                    tma_load_2d(st + off, &m_B, x, (b_lo + bs) * N, full + is_s);
-                    tma_load_2d(st + off + Ly::RAW_BC, &m_C, x, (b_lo + bs) * N, full + is_s);
+                    tma_load_2d(st + off, &m_B, x, (b_lo + bs) * N, full + st_i);
+                    tma_load_2d(st + off + Ly::RAW_BC, &m_C, x, (b_lo + bs) * N, full + st_i);
                 }
-            ++is_;
-            if (++is_s == STAGES) is_s = 0;
-            if (++is_k == ntiles) { is_k = 0; ++is_q; }
+        };
+        // B/C of tile kk (landed in its stage) to fp32 in buffer kk & 1
+        auto convert = [&](int kk) -> bool {
+            if (!__all_sync(0xffffffffu, mbar_wait_sleep(full + kk % STAGES, (kk / STAGES) & 1, p.err, 64)))
+                return false;
+            int b_lo, nb;
+            pass_batches(kk / ntiles, b_lo, nb);
+            const uint8_t *st = smem + (kk % STAGES) * Ly::STAGE + Ly::kBC0;
+            float *dstb = bcf + (kk & 1) * Ly::BCF;
+            constexpr int CH = TT / 4;                      // fp32 chunks per row
+            const int nitems = 2 * nb * N * CH;             // (B or C, batch row, state, chunk)
+            for (int i = lane; i < nitems; i += 32) {
+                const int ch = i % CH, rr = (i / CH) % (nb * N), which = i / (CH * nb * N);
+                const int byte = ch * 4 * (int)sizeof(T);
+                const int pc = byte / Ly::PW, in = byte % Ly::PW;
+                int rch = in >> 4;
+                if constexpr (Ly::SWZ) rch ^= (rr & 7);
+                const uint8_t *src = st + which * Ly::RAW_BC + pc * Ly::PIECE + rr * Ly::PW;
+                float v[4];
+                if constexpr (sizeof(T) == 2) {
+                    const uint2 q2 = *reinterpret_cast<const uint2 *>(src + rch * 16 + (in & 15));
+                    v[0] = __uint_as_float(q2.x << 16); v[1] = __uint_as_float(q2.x & 0xffff0000u);
+                    v[2] = __uint_as_float(q2.y << 16); v[3] = __uint_as_float(q2.y & 0xffff0000u);
+                } else {
+                    const float4 f = *reinterpret_cast<const float4 *>(src + rch * 16);
+                    v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+                }
+                float *drow = dstb + (which * 2 * N + rr) * TT;
+                *reinterpret_cast<float4 *>(drow + bcf_chunk(rr, ch) * 4) = make_float4(v[0], v[1], v[2], v[3]);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bcready + (kk & 1));
+            return true;
         };
         if (lane == 0)
-            while (is_ < STAGES && is_ < total) issue_next();
-        bool ok = true;
-        int q = 0, k = 0, q0 = 0, q1 = 0;
-        for (int kg = 0; kg < total; ++kg) {
-            if (k == 0) pass_rows(q, q0, q1);
+            while (is_ < STAGES && is_ < total) issue(is_++);
+        bool ok = convert(0);
+        for (int kg = 0; ok && kg < total; ++kg) {
+            // B/C of the next tile while the consumers work on this one; its
+            // buffer was last read by tile kg - 1, whose dfull was awaited
+            if (kg + 1 < total && !convert(kg + 1)) break;
             // every consumer is done with tile kg: flush its dB/dC, then refill the stage
-            ok = mbar_wait(dfull + (kg & 1), (kg >> 1) & 1, p.err);
-            ok = __all_sync(0xffffffffu, ok);
+            ok = __all_sync(0xffffffffu, mbar_wait_sleep(dfull + (kg & 1), (kg >> 1) & 1, p.err, 256));
             if (!ok) break;
             {
+                const int q = kg / ntiles, k = kg - q * ntiles;
                 const int t0 = (ntiles - 1 - k) * TT;
-                const int b_lo = q0 / p.dim, nb = (q1 - 1) / p.dim - b_lo + 1;
+                int b_lo, nb;
+                pass_batches(q, b_lo, nb);
                 float *buf = dbc + (kg & 1) * Ly::DBC_PAR;
                 constexpr int QPR = TT / 4;                 // float4 per accumulator row
                 const int nvec = 2 * nb * N * QPR;
                 for (int i = lane; i < nvec; i += 32) {
                     const int tq = i % QPR, n = (i / QPR) % N;
                     const int bs = (i / (QPR * N)) % nb, which = i / (QPR * N * nb);
-                    float *src = buf + ((which * 2 + bs) * N + dbc_row(n)) * DS + tq * 4;
-                    const float4 v = *reinterpret_cast<const float4 *>(src);
-                    *reinterpret_cast<float4 *>(src) = make_float4(0.f, 0.f, 0.f, 0.f);
-                    const int tg = t0 + tq * 4;
+                    const float *src = buf + ((which * 2 + bs) * N + n) * TT;
+                    const int t = tq * 4;
+                    const float4 v = make_float4(src[dbc_col(n, t)], src[dbc_col(n, t + 1)],
+                                                 src[dbc_col(n, t + 2)], src[dbc_col(n, t + 3)]);
+                    const int tg = t0 + t;
                     if (tg < p.L) {
                         float *dst = (which == 0 ? p.dB : p.dC) + ((size_t)(b_lo + bs) * N + n) * p.L + tg;
                         red_add_v4(dst, v);
                     }
                 }
                 __syncwarp();
+                for (int i = lane; i < Ly::DBC_PAR / 4; i += 32)
+                    reinterpret_cast<float4 *>(buf)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+                __syncwarp();
                 if (lane == 0) mbar_arrive(dempty + (kg & 1));
             }
             if (lane == 0 && is_ < total) {
-                ok = mbar_wait(empty + (kg % STAGES), (kg / STAGES) & 1, p.err);
-                if (ok) issue_next();
+                ok = mbar_wait_sleep(empty + (kg % STAGES), (kg / STAGES) & 1, p.err, 64);
+                if (ok) issue(is_++);
             }
             ok = __all_sync(0xffffffffu, ok);
-            if (!ok) break;
-            if (++k == ntiles) { k = 0; ++q; }
         }
         if (lane == 0) {
             // never leave while a copy may still write shared memory
-            for (int kg = (is_ > STAGES ? is_ - STAGES : 0); kg < is_; ++kg)
-                if (!mbar_wait(full + (kg % STAGES), (kg / STAGES) & 1, p.err)) break;
+            for (int kk = (is_ > STAGES ? is_ - STAGES : 0); kk < is_; ++kk)
+                if (!mbar_wait(full + (kk % STAGES), (kk / STAGES) & 1, p.err)) break;
         }
         return;
     }
@@ -271,12 +314,13 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
     float *wP = wbase + Ly::kWp, *wX = wbase + Ly::kWx;
     float *myX = wX + lane * XS;
 
-    float A2[NS], lam[NS], anext[NS], dA_acc[NS];   // A2 = A log2(e)
-    float4 hpre = make_float4(0.f, 0.f, 0.f, 0.f);        // checkpoint of the next window
+    float2 A2p[NS], dA2[NS];                                   // (A log2 e) twice; dA partials
+    float lam[NS], anext[NS];
+    float4 hpre = make_float4(0.f, 0.f, 0.f, 0.f);             // checkpoint of the next window
     float dD_acc = 0.f, db_acc = 0.f, Dd = 0.f, bias_c = 0.f, i_bias = 0.f;
     int row = 0, d = 0, bsel = 0, wb = 0, irow = -1;
     bool live = false, straddle = false;
-    unsigned b1mask = 0;                                   // channels of the second batch row
+    unsigned b1mask = 0;                                       // channels of the second batch row
 
     int s = 0, phase = 0, q = 0, k = 0, q0 = 0, q1 = 0;
     for (int kg = 0; kg < total; ++kg) {
@@ -294,10 +338,11 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
             wb = b1mask != 0 ? 1 : 0;
 #pragma unroll
             for (int j = 0; j < NS; ++j) {
-                A2[j] = live ? p.A[(size_t)d * N + g * NS + j] * SSM_LOG2E : 0.f;
+                const float a2 = live ? p.A[(size_t)d * N + g * NS + j] * SSM_LOG2E : 0.f;
+                A2p[j] = make_float2(a2, a2);
+                dA2[j] = make_float2(0.f, 0.f);
                 lam[j] = 0.f;
                 anext[j] = 1.f;
-                dA_acc[j] = 0.f;
             }
             Dd = (live && p.D) ? p.D[d] : 0.f;
             bias_c = (live && p.delta_bias) ? p.delta_bias[d] : 0.f;
@@ -308,14 +353,14 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
             db_acc = 0.f;
             // starting state of the first window visited (the one holding step L-1)
             const int kc0 = (p.L - 1) / W - 1;
-            hpre = (live && kc0 >= 0) ? __ldg(reinterpret_cast<const float4 *>(
-                                            p.ckpt + ((size_t)row * p.n_ckpt + kc0) * N + g * NS))
+            hpre = (live && kc0 >= 0) ? ldg_f4_now(p.ckpt + ((size_t)row * p.n_ckpt + kc0) * N + g * NS)
                                       : make_float4(0.f, 0.f, 0.f, 0.f);
         }
         const int wrow0 = q0 + warp * CPW;
         {
             // every lane waits; the warp leaves together if any wait gave up
             bool ok = mbar_wait(full + s, phase, p.err);
+            ok = ok && mbar_wait(bcready + (kg & 1), (kg >> 1) & 1, p.err);
             if (kg >= 2) ok = ok && mbar_wait(dempty + (kg & 1), ((kg - 2) >> 1) & 1, p.err);
             if (!__all_sync(0xffffffffu, ok)) return;
         }
@@ -338,14 +383,14 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                     IO<T>::unpack(*reinterpret_cast<const uint4 *>(rawD + o), dr);
                     IO<T>::unpack(*reinterpret_cast<const uint4 *>(rawU + o), uu);
                     IO<T>::unpack(*reinterpret_cast<const uint4 *>(rawG + o), gg);
-                    if (p.has_z) IO<T>::unpack(*reinterpret_cast<const uint4 *>(rawZ + o), zz);
+                    if constexpr (HZ) IO<T>::unpack(*reinterpret_cast<const uint4 *>(rawZ + o), zz);
 #pragma unroll
                     for (int e = 0; e < V; ++e) {
                         const bool ok = irow >= 0 && (t0 + it_t + v0 + e) < p.L;
                         const float r = dr[e] + i_bias;
-                        const float dtv = p.softplus ? softplus_fast(r) : r;
+                        const float dtv = SP ? softplus_fast(r) : r;
                         float gyv = gg[e];
-                        if (p.has_z) gyv *= zz[e] * sigmoid(zz[e]);
+                        if constexpr (HZ) gyv *= zz[e] * sigmoid(zz[e]);
                         dt[v0 + e] = ok ? dtv : 0.f;
                         du[v0 + e] = ok ? dtv * uu[e] : 0.f;
                         gy[v0 + e] = ok ? gyv : 0.f;
@@ -362,45 +407,54 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
             }
             __syncwarp();
 
-            const uint8_t *rawB = st + Ly::kBC0;
-            const uint8_t *rawC = rawB + Ly::RAW_BC;
-            auto bc_chunk = [&](const uint8_t *base, int rr, int tb) -> uint4 {
-                const int byte = tb * (int)sizeof(T);
-                const int pc = byte / Ly::PW, in = byte % Ly::PW;
-                int chunk = in >> 4;
-                if constexpr (Ly::SWZ) chunk ^= (rr & 7);
-                return *reinterpret_cast<const uint4 *>(base + pc * Ly::PIECE + rr * Ly::PW + (chunk << 4));
+            const float *bcfB = bcf + (kg & 1) * Ly::BCF + bsel * N * TT;
+            const float *bcfC = bcfB + 2 * N * TT;
+            const int swz = (bsel * 4 + g) & 7;              // bcf_chunk of this lane's rows
+            auto bc4 = [&](const float *base, int j, int tb) -> float4 {
+                return *reinterpret_cast<const float4 *>(base + (g * NS + j) * TT + (((tb >> 2) ^ swz) << 2));
             };
-            const int rr0 = bsel * N + g * NS;
-            // Sum of the transpose buffer over the quarter-warp's channels for
-            // step c of the window, states 4g..4g+3, added to the tile
-            // accumulator `which` (0: dB, 1: dC).
+            // Sum of the transpose buffer over the quarter-warp's 8 channels:
+            // lane (g, c) takes state 4g + c/2, steps 4(c&1)..4(c&1)+3 of the
+            // window, and adds them to accumulator `which` (0: dB, 1: dC).
             auto reduce_x = [&](int which, int tw) {
                 __syncwarp();
-                float4 s0 = make_float4(0.f, 0.f, 0.f, 0.f), s1 = s0;
+                const float *src = wX + g * CPW * XS + c * 4;
+                const int n = g * NS + (c >> 1), tb = tw + (c & 1) * 4;
+                float *dst = dbuf + (which * 2 * N + n) * TT;
+                if (!straddle) {
+                    float4 s0 = *reinterpret_cast<const float4 *>(src);
 #pragma unroll
-                for (int cc = 0; cc < CPW; ++cc) {
-                    const float4 v = *reinterpret_cast<const float4 *>(wX + (g * CPW + cc) * XS + c * NS);
-                    if (straddle && ((b1mask >> cc) & 1)) s1 = f4add(s1, v);
-                    else s0 = f4add(s0, v);
-                }
-                __syncwarp();
-                float *dst = dbuf + ((which * 2 + (straddle ? 0 : wb)) * N) * DS + tw + c;
-                atomicAdd(dst + dbc_row(g * NS + 0) * DS, s0.x);
-                atomicAdd(dst + dbc_row(g * NS + 1) * DS, s0.y);
-                atomicAdd(dst + dbc_row(g * NS + 2) * DS, s0.z);
-                atomicAdd(dst + dbc_row(g * NS + 3) * DS, s0.w);
-                if (straddle) {
-                    dst += N * DS;
-                    atomicAdd(dst + dbc_row(g * NS + 0) * DS, s1.x);
-                    atomicAdd(dst + dbc_row(g * NS + 1) * DS, s1.y);
-                    atomicAdd(dst + dbc_row(g * NS + 2) * DS, s1.z);
-                    atomicAdd(dst + dbc_row(g * NS + 3) * DS, s1.w);
+                    for (int cc = 1; cc < CPW; ++cc) s0 = f4add(s0, *reinterpret_cast<const float4 *>(src + cc * XS));
+                    __syncwarp();
+                    dst += wb * N * TT;
+                    atomicAdd(dst + dbc_col(n, tb + 0), s0.x);
+                    atomicAdd(dst + dbc_col(n, tb + 1), s0.y);
+                    atomicAdd(dst + dbc_col(n, tb + 2), s0.z);
+                    atomicAdd(dst + dbc_col(n, tb + 3), s0.w);
+                } else {
+                    // channels of two batch rows: one sum per batch row
+                    float4 s0 = make_float4(0.f, 0.f, 0.f, 0.f), s1 = s0;
+#pragma unroll
+                    for (int cc = 0; cc < CPW; ++cc) {
+                        const float4 v = *reinterpret_cast<const float4 *>(src + cc * XS);
+                        if ((b1mask >> cc) & 1) s1 = f4add(s1, v);
+                        else s0 = f4add(s0, v);
+                    }
+                    __syncwarp();
+                    atomicAdd(dst + dbc_col(n, tb + 0), s0.x);
+                    atomicAdd(dst + dbc_col(n, tb + 1), s0.y);
+                    atomicAdd(dst + dbc_col(n, tb + 2), s0.z);
+                    atomicAdd(dst + dbc_col(n, tb + 3), s0.w);
+                    dst += N * TT;
+                    atomicAdd(dst + dbc_col(n, tb + 0), s1.x);
+                    atomicAdd(dst + dbc_col(n, tb + 1), s1.y);
+                    atomicAdd(dst + dbc_col(n, tb + 2), s1.z);
+                    atomicAdd(dst + dbc_col(n, tb + 3), s1.w);
                 }
             };
 
             // (2) 8-step windows, last to first
-#pragma unroll 1
+#pragma unroll kWinUnroll
             for (int w = Ly::NWIN - 1; w >= 0; --w) {
                 const int tw = w * W;                       // window start within the tile
                 const int tgw = t0 + tw;                    // and within the sequence
@@ -408,88 +462,91 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                 float h[NS] = {hpre.x, hpre.y, hpre.z, hpre.w};
                 {
                     const int kc = tgw / W - 2;             // checkpoint of the next window
-                    hpre = (live && kc >= 0) ? __ldg(reinterpret_cast<const float4 *>(
-                                                   p.ckpt + ((size_t)row * p.n_ckpt + kc) * N + g * NS))
+                    hpre = (live && kc >= 0) ? ldg_f4_now(p.ckpt + ((size_t)row * p.n_ckpt + kc) * N + g * NS)
                                              : make_float4(0.f, 0.f, 0.f, 0.f);
                 }
-                BCWin<T> Bw[NS], Cw[NS];
+                // Forward recompute over pairs of steps (f32x2 arithmetic):
+                // Ā_t, Ā_t h_{t-1}, the y partials and gy h_t (for dC).
+                float2 ab2[W / 2][NS], ahp2[W / 2][NS];
 #pragma unroll
-                for (int j = 0; j < NS; ++j) {
-                    if constexpr (sizeof(T) == 2) {
-                        Bw[j].v = bc_chunk(rawB, rr0 + j, tw);
-                        Cw[j].v = bc_chunk(rawC, rr0 + j, tw);
-                    } else {
-                        Bw[j].v[0] = bc_chunk(rawB, rr0 + j, tw);
-                        Bw[j].v[1] = bc_chunk(rawB, rr0 + j, tw + 4);
-                        Cw[j].v[0] = bc_chunk(rawC, rr0 + j, tw);
-                        Cw[j].v[1] = bc_chunk(rawC, rr0 + j, tw + 4);
-                    }
-                }
-                // forward recompute, 4 steps at a time: Ā_t, Ā_t h_{t-1}, the y
-                // partials, and gy h_t for dC
-                float ab[W][NS], ahp[W][NS];
-                float *pY = wP + (0 * NT + g) * CPW * PS + c * PS;
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int tb = tw + 4 * hh;
+                    const float4 dt4 = *reinterpret_cast<const float4 *>(wDt + c * WS + tb);
+                    const float4 du4 = *reinterpret_cast<const float4 *>(wDu + c * WS + tb);
+                    const float4 gy4 = *reinterpret_cast<const float4 *>(wGy + c * WS + tb);
+                    const float2 dtp[2] = {make_float2(dt4.x, dt4.y), make_float2(dt4.z, dt4.w)};
+                    const float2 dup[2] = {make_float2(du4.x, du4.y), make_float2(du4.z, du4.w)};
+                    const float2 gyp[2] = {make_float2(gy4.x, gy4.y), make_float2(gy4.z, gy4.w)};
+                    float2 y2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-                for (int t4 = 0; t4 < W; t4 += 4) {
-                    const float4 dt4 = *reinterpret_cast<const float4 *>(wDt + c * WS + tw + t4);
-                    const float4 du4 = *reinterpret_cast<const float4 *>(wDu + c * WS + tw + t4);
-                    const float4 gy4 = *reinterpret_cast<const float4 *>(wGy + c * WS + tw + t4);
-                    const float dt[4] = {dt4.x, dt4.y, dt4.z, dt4.w}, du[4] = {du4.x, du4.y, du4.z, du4.w};
-                    const float gy[4] = {gy4.x, gy4.y, gy4.z, gy4.w};
-                    float yp[4];
+                    for (int j = 0; j < NS; ++j) {
+                        const float4 B4 = bc4(bcfB, j, tb), C4 = bc4(bcfC, j, tb);
+                        const float2 Bp[2] = {make_float2(B4.x, B4.y), make_float2(B4.z, B4.w)};
+                        const float2 Cp[2] = {make_float2(C4.x, C4.y), make_float2(C4.z, C4.w)};
+                        float2 xc[2];
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int t = t4 + i;
-                        float acc = 0.f, xc[NS];
-#pragma unroll
-                        for (int j = 0; j < NS; ++j) {
-                            const float a = ex2(dt[i] * A2[j]);
-                            ab[t][j] = a;
-                            ahp[t][j] = a * h[j];
-                            h[j] = fmaf(du[i], Bw[j].at(t), ahp[t][j]);
-                            acc = fmaf(Cw[j].at(t), h[j], acc);
-                            xc[j] = gy[i] * h[j];
+                        for (int pp = 0; pp < 2; ++pp) {
+                            const int P = 2 * hh + pp;
+                            const float2 arg = __fmul2_rn(dtp[pp], A2p[j]);
+                            const float2 a = make_float2(ex2(arg.x), ex2(arg.y));
+                            const float2 beta = __fmul2_rn(dup[pp], Bp[pp]);
+                            const float h0 = fmaf(a.x, h[j], beta.x);
+                            const float h1 = fmaf(a.y, h0, beta.y);
+                            h[j] = h1;
+                            const float2 hv = make_float2(h0, h1);
+                            ab2[P][j] = a;
+                            ahp2[P][j] = __ffma2_rn(beta, make_float2(-1.f, -1.f), hv);   // Ā_t h_{t-1}
+                            y2[pp] = __ffma2_rn(Cp[pp], hv, y2[pp]);
+                            xc[pp] = __fmul2_rn(gyp[pp], hv);
                         }
-                        yp[i] = acc;
-                        *reinterpret_cast<float4 *>(myX + t * NS) = make_float4(xc[0], xc[1], xc[2], xc[3]);
+                        *reinterpret_cast<float4 *>(myX + (2 * j + hh) * 4) =
+                            make_float4(xc[0].x, xc[0].y, xc[1].x, xc[1].y);
                     }
-                    *reinterpret_cast<float4 *>(pY + t4) = make_float4(yp[0], yp[1], yp[2], yp[3]);
+                    *reinterpret_cast<float4 *>(wP + (0 * NT + g) * CPW * PS + c * PS + 4 * hh) =
+                        make_float4(y2[0].x, y2[0].y, y2[1].x, y2[1].y);
                 }
                 reduce_x(1, tw);
-                // reverse sweep, 4 steps at a time.  The A-weighted sum is kept
-                // in units of A log2(e) and rescaled per element.
-                float *pA = wP + (1 * NT + g) * CPW * PS + c * PS;
-                float *pB = wP + (2 * NT + g) * CPW * PS + c * PS;
+                // Reverse sweep over pairs of steps.  The A-weighted sum is
+                // kept in units of A log2(e) and rescaled per element.
 #pragma unroll
-                for (int t4 = W - 4; t4 >= 0; t4 -= 4) {
-                    const float4 dt4 = *reinterpret_cast<const float4 *>(wDt + c * WS + tw + t4);
-                    const float4 du4 = *reinterpret_cast<const float4 *>(wDu + c * WS + tw + t4);
-                    const float4 gy4 = *reinterpret_cast<const float4 *>(wGy + c * WS + tw + t4);
-                    const float dt[4] = {dt4.x, dt4.y, dt4.z, dt4.w}, du[4] = {du4.x, du4.y, du4.z, du4.w};
-                    const float gy[4] = {gy4.x, gy4.y, gy4.z, gy4.w};
-                    float sa[4], sb[4];
+                for (int hh = 1; hh >= 0; --hh) {
+                    const int tb = tw + 4 * hh;
+                    const float4 dt4 = *reinterpret_cast<const float4 *>(wDt + c * WS + tb);
+                    const float4 du4 = *reinterpret_cast<const float4 *>(wDu + c * WS + tb);
+                    const float4 gy4 = *reinterpret_cast<const float4 *>(wGy + c * WS + tb);
+                    const float2 dtp[2] = {make_float2(dt4.x, dt4.y), make_float2(dt4.z, dt4.w)};
+                    const float2 dup[2] = {make_float2(du4.x, du4.y), make_float2(du4.z, du4.w)};
+                    const float2 gyp[2] = {make_float2(gy4.x, gy4.y), make_float2(gy4.z, gy4.w)};
+                    float2 sa2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+                    float2 sb2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-                    for (int i = 3; i >= 0; --i) {
-                        const int t = t4 + i;
-                        float a_sa = 0.f, a_sb = 0.f, xb[NS];
+                    for (int j = 0; j < NS; ++j) {
+                        const float4 B4 = bc4(bcfB, j, tb), C4 = bc4(bcfC, j, tb);
+                        const float2 Bp[2] = {make_float2(B4.x, B4.y), make_float2(B4.z, B4.w)};
+                        const float2 Cp[2] = {make_float2(C4.x, C4.y), make_float2(C4.z, C4.w)};
+                        float2 xb[2];
 #pragma unroll
-                        for (int j = 0; j < NS; ++j) {
-                            const float Bt = Bw[j].at(t);
-                            const float l = fmaf(anext[j], lam[j], Cw[j].at(t) * gy[i]);
-                            const float wv = l * ahp[t][j];
-                            dA_acc[j] = fmaf(dt[i], wv, dA_acc[j]);
-                            a_sa = fmaf(A2[j], wv, a_sa);
-                            a_sb = fmaf(l, Bt, a_sb);
-                            xb[j] = l * du[i];
-                            lam[j] = l;
-                            anext[j] = ab[t][j];
+                        for (int pp = 1; pp >= 0; --pp) {
+                            const int P = 2 * hh + pp;
+                            const float2 cg = __fmul2_rn(Cp[pp], gyp[pp]);
+                            const float l1 = fmaf(anext[j], lam[j], cg.y);      // λ of the later step
+                            const float l0 = fmaf(ab2[P][j].y, l1, cg.x);       // λ of the earlier step
+                            const float2 l2 = make_float2(l0, l1);
+                            const float2 wv = __fmul2_rn(l2, ahp2[P][j]);
+                            dA2[j] = __ffma2_rn(dtp[pp], wv, dA2[j]);
+                            sa2[pp] = __ffma2_rn(A2p[j], wv, sa2[pp]);
+                            sb2[pp] = __ffma2_rn(l2, Bp[pp], sb2[pp]);
+                            xb[pp] = __fmul2_rn(l2, dup[pp]);
+                            lam[j] = l0;
+                            anext[j] = ab2[P][j].x;
                         }
-                        sa[i] = a_sa;
-                        sb[i] = a_sb;
-                        *reinterpret_cast<float4 *>(myX + t * NS) = make_float4(xb[0], xb[1], xb[2], xb[3]);
+                        *reinterpret_cast<float4 *>(myX + (2 * j + hh) * 4) =
+                            make_float4(xb[0].x, xb[0].y, xb[1].x, xb[1].y);
                     }
-                    *reinterpret_cast<float4 *>(pA + t4) = make_float4(sa[0], sa[1], sa[2], sa[3]);
-                    *reinterpret_cast<float4 *>(pB + t4) = make_float4(sb[0], sb[1], sb[2], sb[3]);
+                    *reinterpret_cast<float4 *>(wP + (1 * NT + g) * CPW * PS + c * PS + 4 * hh) =
+                        make_float4(sa2[0].x, sa2[0].y, sa2[1].x, sa2[1].y);
+                    *reinterpret_cast<float4 *>(wP + (2 * NT + g) * CPW * PS + c * PS + 4 * hh) =
+                        make_float4(sb2[0].x, sb2[0].y, sb2[1].x, sb2[1].y);
                 }
                 reduce_x(0, tw);   // its leading __syncwarp also publishes the partials
                 // per-element results: lane (g, c) finishes steps 2g and 2g+1 of channel c
@@ -514,13 +571,13 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                     float dzv[2] = {0.f, 0.f}, duv[2], ddv[2];
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
-                        if (p.has_z) {
+                        if constexpr (HZ) {
                             const float zz = IO<T>::to_f(rawZ[o + e]);
                             const float sg = sigmoid(zz);
                             dzv[e] = gv[e] * yy[e] * sg * fmaf(zz, 1.f - sg, 1.f);
                         }
                         const float dDelta = fmaf(x[e], sb2[e], sa2[e]);
-                        ddv[e] = p.softplus ? dDelta * sigmoid(IO<T>::to_f(rawD[o + e]) + bias_c) : dDelta;
+                        ddv[e] = SP ? dDelta * sigmoid(IO<T>::to_f(rawD[o + e]) + bias_c) : dDelta;
                         duv[e] = fmaf(gy2[e], Dd, dt2[e] * sb2[e]);
                         dD_acc = fmaf(gy2[e], x[e], dD_acc);
                         db_acc += ddv[e];
@@ -528,7 +585,7 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                     const size_t off = (size_t)row * p.L + tgw + t;
                     __stcs(reinterpret_cast<float2 *>(p.du + off), make_float2(duv[0], duv[1]));
                     __stcs(reinterpret_cast<float2 *>(p.ddelta + off), make_float2(ddv[0], ddv[1]));
-                    if (p.has_z) __stcs(reinterpret_cast<float2 *>(p.dz + off), make_float2(dzv[0], dzv[1]));
+                    if constexpr (HZ) __stcs(reinterpret_cast<float2 *>(p.dz + off), make_float2(dzv[0], dzv[1]));
                 }
                 __syncwarp();   // wP and the transpose buffer are rewritten by the next window
             }
@@ -543,7 +600,7 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
             // end of a pass over this CTA's rows: per-channel sums
             if (live) {
 #pragma unroll
-                for (int j = 0; j < NS; ++j) atomicAdd(p.dA + (size_t)d * N + g * NS + j, dA_acc[j]);
+                for (int j = 0; j < NS; ++j) atomicAdd(p.dA + (size_t)d * N + g * NS + j, dA2[j].x + dA2[j].y);
             }
 #pragma unroll
             for (int m = CPW; m < 32; m <<= 1) {    // lanes c, c+8, c+16, c+24 share channel c
@@ -598,7 +655,7 @@ int bwd_sm_count() {
     return count[dev];
 }
 
-template <typename T, int NWC, int STAGES>
+template <typename T, int NWC, int STAGES, bool HZ, bool SP>
 cudaError_t launch_bwd_tma_cfg(const BwdParams &bp, int rows_max, cudaStream_t stream) {
     using Ly = BwdLayout<T, NWC, STAGES>;
     const int P = bp.batch * bp.dim;
@@ -621,7 +678,7 @@ cudaError_t launch_bwd_tma_cfg(const BwdParams &bp, int rows_max, cudaStream_t s
     p.softplus = bp.softplus; p.has_z = bp.z != nullptr; p.rows_max = rows_max;
     p.err = device_error_word();
     if (!p.err) return cudaErrorInvalidDevice;
-    auto kern = bwd_tma_kernel<T, NWC, STAGES>;
+    auto kern = bwd_tma_kernel<T, NWC, STAGES, HZ, SP>;
     static bool attr_done = false;
     if (!attr_done) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Ly::kAlloc);
@@ -630,6 +687,16 @@ cudaError_t launch_bwd_tma_cfg(const BwdParams &bp, int rows_max, cudaStream_t s
     }
     kern<<<grid, Ly::kThreads, Ly::kAlloc, stream>>>(md, mu, mz, mg, mB, mC, p);
     return cudaGetLastError();
+}
+
+// The gate and the softplus are compile-time switches of the kernel.
+template <typename T, int NWC>
+cudaError_t launch_bwd_tma_flags(const BwdParams &bp, int rows_max, cudaStream_t stream) {
+    const bool hz = bp.z != nullptr, sp = bp.softplus != 0;
+    if (hz && sp) return launch_bwd_tma_cfg<T, NWC, 2, true, true>(bp, rows_max, stream);
+    if (hz) return launch_bwd_tma_cfg<T, NWC, 2, true, false>(bp, rows_max, stream);
+    if (sp) return launch_bwd_tma_cfg<T, NWC, 2, false, true>(bp, rows_max, stream);
+    return launch_bwd_tma_cfg<T, NWC, 2, false, false>(bp, rows_max, stream);
 }
 
 bool aligned_to(const void *ptr, uintptr_t a) { return (reinterpret_cast<uintptr_t>(ptr) % a) == 0; }
@@ -663,8 +730,8 @@ bool try_launch_bwd_tma(const BwdParams &bp, cudaStream_t stream, cudaError_t *e
     const long long npass = (R + cap - 1) / cap;
     const long long rows_max = (R + npass - 1) / npass;
     if (rows_max > bp.dim) return false;   // a pass spans at most two batch rows
-    *err = bp.io_bf16 ? launch_bwd_tma_cfg<__nv_bfloat16, kBwdWarpsBf16, 2>(bp, (int)rows_max, stream)
-                      : launch_bwd_tma_cfg<float, kBwdWarpsF32, 2>(bp, (int)rows_max, stream);
+    *err = bp.io_bf16 ? launch_bwd_tma_flags<__nv_bfloat16, kBwdWarpsBf16>(bp, (int)rows_max, stream)
+                      : launch_bwd_tma_flags<float, kBwdWarpsF32>(bp, (int)rows_max, stream);
     return true;
 }
 

@@ -197,7 +197,7 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
         int s = 0, phase = 0, q = 0, tile = 0, q0 = 0, q1 = 0, b_lo = 0, nb = 1;
         for (; issued < total && ok; ++issued) {
             if (issued >= STAGES) {   // wait until every consumer left this stage
-                ok = mbar_wait(empty + s, phase ^ 1, p.err);
+                ok = mbar_wait_sleep(empty + s, phase ^ 1, p.err, 64);
                 if (!ok) break;
             }
             if (tile == 0) {

@@ -67,6 +67,24 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *e
     return true;
 }
 
+// As mbar_wait, but sleeps about `ns` nanoseconds between polls.  For a warp
+// whose waits are normally long (a producer waiting for the consumers to
+// finish a tile): polling without a pause would take issue slots from the
+// warps that do the work.
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t *bar, uint32_t parity, int *err,
+                                                unsigned ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        __nanosleep(ns);
+        if (clock64() - t0 > kWaitBudgetCycles) {
+            atomicExch(err, kErrWaitTimeout);
+            return false;
+        }
+    }
+    return true;
+}
+
 // 2-D tiled TMA load of box {x..x+bx, y..y+by} into shared memory; completion
 // is signalled on `bar` as transaction bytes.  Out-of-range elements read 0.
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y,
