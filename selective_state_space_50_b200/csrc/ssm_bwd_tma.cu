@@ -619,56 +619,21 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
 
 // ------------------------------------------------------------------ host side
 
-PFN_cuTensorMapEncodeTiled_v12000 bwd_get_encode() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult qr;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qr) == cudaSuccess &&
-            qr == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    }
-    return fn;
-}
-
-bool bwd_make_map(CUtensorMap *m, const void *base, bool bf16, uint64_t rows, uint64_t cols,
-                  uint32_t box_cols, uint32_t box_rows, bool swizzle128) {
-    auto enc = bwd_get_encode();
-    if (!enc) return false;
-    const uint64_t es = bf16 ? 2 : 4;
-    cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols * es};
-    cuuint32_t box[2] = {box_cols, box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    return enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
-               const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-               swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-int bwd_sm_count() {
-    static int count[64] = {0};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64) return 148;
-    if (!count[dev]) cudaDeviceGetAttribute(&count[dev], cudaDevAttrMultiProcessorCount, dev);
-    return count[dev];
-}
 
 template <typename T, int NWC, int STAGES, bool HZ, bool SP>
 cudaError_t launch_bwd_tma_cfg(const BwdParams &bp, int rows_max, cudaStream_t stream) {
     using Ly = BwdLayout<T, NWC, STAGES>;
     const int P = bp.batch * bp.dim;
-    const int grid = std::min(bwd_sm_count(), P);
+    const int grid = std::min(device_sm_count(), P);
     const bool bf16 = sizeof(T) == 2;
     CUtensorMap md, mu, mz, mg, mB, mC;
     const uint32_t bc_box = Ly::PW / sizeof(T);
-    if (!bwd_make_map(&md, bp.delta, bf16, P, bp.L, Ly::TT, rows_max, false) ||
-        !bwd_make_map(&mu, bp.u, bf16, P, bp.L, Ly::TT, rows_max, false) ||
-        !bwd_make_map(&mz, bp.z ? bp.z : bp.u, bf16, P, bp.L, Ly::TT, rows_max, false) ||
-        !bwd_make_map(&mg, bp.dout, bf16, P, bp.L, Ly::TT, rows_max, false) ||
-        !bwd_make_map(&mB, bp.B, bf16, (uint64_t)bp.batch * Ly::N, bp.L, bc_box, Ly::N, Ly::SWZ) ||
-        !bwd_make_map(&mC, bp.C, bf16, (uint64_t)bp.batch * Ly::N, bp.L, bc_box, Ly::N, Ly::SWZ))
+    if (!make_tma_map_2d(&md, bp.delta, bf16, P, bp.L, Ly::TT, rows_max, false) ||
+        !make_tma_map_2d(&mu, bp.u, bf16, P, bp.L, Ly::TT, rows_max, false) ||
+        !make_tma_map_2d(&mz, bp.z ? bp.z : bp.u, bf16, P, bp.L, Ly::TT, rows_max, false) ||
+        !make_tma_map_2d(&mg, bp.dout, bf16, P, bp.L, Ly::TT, rows_max, false) ||
+        !make_tma_map_2d(&mB, bp.B, bf16, (uint64_t)bp.batch * Ly::N, bp.L, bc_box, Ly::N, Ly::SWZ) ||
+        !make_tma_map_2d(&mC, bp.C, bf16, (uint64_t)bp.batch * Ly::N, bp.L, bc_box, Ly::N, Ly::SWZ))
         return cudaErrorInvalidValue;
     TmaBwdParams p{};
     p.A = bp.A; p.D = bp.D; p.delta_bias = bp.delta_bias; p.ckpt = bp.ckpt;
@@ -721,9 +686,9 @@ bool try_launch_bwd_tma(const BwdParams &bp, cudaStream_t stream, cudaError_t *e
     if (!aligned_to(bp.ckpt, 16) || !aligned_to(bp.dB, 16) || !aligned_to(bp.dC, 16) ||
         !aligned_to(bp.du, 8) || !aligned_to(bp.ddelta, 8) || (bp.dz && !aligned_to(bp.dz, 8)))
         return false;
-    if (!bwd_get_encode()) return false;
+    if (!tma_available()) return false;
     const long long P = (long long)bp.batch * bp.dim;
-    const int sms = bwd_sm_count();
+    const int sms = device_sm_count();
     if (P < sms) return false;
     const long long cap = (bp.io_bf16 ? kBwdWarpsBf16 : kBwdWarpsF32) * 8;
     const long long R = (P + sms - 1) / sms;

@@ -259,8 +259,8 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
             live = row < q1;
             const int d = live ? row % p.dim : 0;
             bsel = live ? row / p.dim - q0 / p.dim : 0;
-#pragma unroll
             bool neg = true;
+#pragma unroll
             for (int j = 0; j < NS; ++j) {
                 const float a = live ? p.A[(size_t)d * N + g * NS + j] * SSM_LOG2E : 0.f;
                 A2d[j] = make_float2(a, a);
@@ -454,60 +454,22 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
 
 // ------------------------------------------------------------------ host side
 
-PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    }
-    return fn;
-}
-
-bool make_map(CUtensorMap *m, const void *base, bool bf16, uint64_t rows, uint64_t cols, uint32_t box_cols,
-              uint32_t box_rows, bool swizzle128 = false) {
-    auto enc = get_encode();
-    if (!enc) return false;
-    const uint64_t es = bf16 ? 2 : 4;
-    cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols * es};
-    cuuint32_t box[2] = {box_cols, box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
-                     const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                     swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
-                     CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
-int sm_count() {
-    static int count[64] = {0};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64) return 148;
-    if (!count[dev]) cudaDeviceGetAttribute(&count[dev], cudaDevAttrMultiProcessorCount, dev);
-    return count[dev];
-}
 
 template <typename T, int NT, int NS, int TT, int NWC, int STAGES>
 cudaError_t launch_cfg(const FwdParams &fp, cudaStream_t stream) {
     using Ly = TmaLayout<T, NT, NS, TT, NWC, STAGES>;
     const int P = fp.batch * fp.dim;
-    const int grid = std::min(sm_count(), P);
+    const int grid = std::min(device_sm_count(), P);
     const int R = (P + grid - 1) / grid;
     const int npass = (R + Ly::MAXR - 1) / Ly::MAXR;
     const int rows_max = (R + npass - 1) / npass;
     const bool bf16 = sizeof(T) == 2;
     CUtensorMap md, mu, mz, mB, mC;
-    if (!make_map(&md, fp.delta, bf16, P, fp.L, TT, rows_max) ||
-        !make_map(&mu, fp.u, bf16, P, fp.L, TT, rows_max) ||
-        !make_map(&mz, fp.z ? fp.z : fp.u, bf16, P, fp.L, TT, rows_max) ||
-        !make_map(&mB, fp.B, bf16, (uint64_t)fp.batch * fp.N, fp.L, Ly::PW / sizeof(T), Ly::N, Ly::SWZ) ||
-        !make_map(&mC, fp.C, bf16, (uint64_t)fp.batch * fp.N, fp.L, Ly::PW / sizeof(T), Ly::N, Ly::SWZ))
+    if (!make_tma_map_2d(&md, fp.delta, bf16, P, fp.L, TT, rows_max, false) ||
+        !make_tma_map_2d(&mu, fp.u, bf16, P, fp.L, TT, rows_max, false) ||
+        !make_tma_map_2d(&mz, fp.z ? fp.z : fp.u, bf16, P, fp.L, TT, rows_max, false) ||
+        !make_tma_map_2d(&mB, fp.B, bf16, (uint64_t)fp.batch * fp.N, fp.L, Ly::PW / sizeof(T), Ly::N, Ly::SWZ) ||
+        !make_tma_map_2d(&mC, fp.C, bf16, (uint64_t)fp.batch * fp.N, fp.L, Ly::PW / sizeof(T), Ly::N, Ly::SWZ))
         return cudaErrorInvalidValue;
     TmaFwdParams p{};
     p.A = fp.A; p.D = fp.D; p.delta_bias = fp.delta_bias; p.out = fp.out;
@@ -612,9 +574,9 @@ bool nt_valid(int N, int nt) {
 bool try_launch_fwd_tma(const FwdParams &fp, cudaStream_t stream, cudaError_t *err) {
     if (!fp.vec_ok || !fp.out) return false;
     if (fp.N != 8 && fp.N != 16 && fp.N != 32) return false;
-    if (!get_encode()) return false;
+    if (!tma_available()) return false;
     const long long P = (long long)fp.batch * fp.dim;
-    const int sms = sm_count();
+    const int sms = device_sm_count();
     if (P < sms) return false;                      // fewer channels than SMs
     const long long R = (P + sms - 1) / sms;        // rows per SM
     // Lane split: the fewest lanes per channel that still give every SM

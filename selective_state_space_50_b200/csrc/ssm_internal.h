@@ -1,7 +1,9 @@
 // Internal launch interface between the C ABI (ssm_api.cu) and the kernels.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
+#include <stdint.h>
 
 #include "ssm_scan.h"
 
@@ -56,6 +58,15 @@ int *device_error_word();
 // clears it when set.
 cudaError_t read_and_clear_device_error(int *value, cudaStream_t stream);
 cudaError_t launch_bwd(const BwdParams &p, cudaStream_t stream);
+
+// TMA host helpers (ssm_tma_host.cu).  tma_available() is false when the
+// driver does not expose the tensor-map encoder.  make_tma_map_2d describes a
+// row-major [rows x cols] bf16 or fp32 array with a [box_rows x box_cols] box
+// (128-byte swizzle on request).  device_sm_count() caches per device.
+bool tma_available();
+bool make_tma_map_2d(CUtensorMap *m, const void *base, bool bf16, uint64_t rows, uint64_t cols,
+                     uint32_t box_cols, uint32_t box_rows, bool swizzle128);
+int device_sm_count();
 // Launches the TMA-fed persistent backward when it applies (dstate 16, 16-byte
 // aligned rows and checkpoints, at least one channel row per SM); returns
 // false when the general backward must be used.  SSM_BWD_KERNEL=general in
