@@ -250,13 +250,19 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
 
     int s = 0, phase = 0;          // ring slot and its parity for tile kg
     int q = 0, tile = 0, q0 = 0, q1 = 0;
+    int rpw = CPW;                 // rows per warp in this pass (the same for every warp, +-1 row)
     for (int kg = 0; kg < total; ++kg) {
-        if (tile == 0) pass_rows(q, q0, q1);
+        if (tile == 0) {
+            pass_rows(q, q0, q1);
+            // spread the pass's rows evenly over the warps
+            rpw = (q1 - q0 + NWC - 1) / NWC;
+        }
         const int t0 = tile * TT;
-        const int wrow0 = q0 + warp * CPW;   // first row of this warp in the pass
+        const int wrow0 = q0 + warp * rpw;   // first row of this warp in the pass
+        const int wend = min(wrow0 + rpw, q1);
         if (tile == 0) {
             const int row = wrow0 + c;
-            live = row < q1;
+            live = row < wend;
             const int d = live ? row % p.dim : 0;
             bsel = live ? row / p.dim - q0 / p.dim : 0;
             bool neg = true;
@@ -271,7 +277,7 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
 #pragma unroll
             for (int i = 0; i < IPL; ++i) {
                 const int rr = wrow0 + (lane + 32 * i) / CPR;
-                const bool ok = rr < q1;
+                const bool ok = rr < wend;
                 const int dd = ok ? rr % p.dim : 0;
                 irow[i] = ok ? rr : -1;
                 Dd[i] = (ok && p.D) ? p.D[dd] : 0.f;
@@ -281,11 +287,11 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
         // every lane waits; the warp leaves together if any wait gave up
         if (!__all_sync(0xffffffffu, mbar_wait(full + s, phase, p.err))) return;
 
-        if (wrow0 < q1) {
+        if (wrow0 < wend) {
             const uint8_t *st = smem + s * Ly::STAGE;
-            const T *rawD = reinterpret_cast<const T *>(st) + warp * CPW * TT;
-            const T *rawU = reinterpret_cast<const T *>(st + Ly::RAW_CH) + warp * CPW * TT;
-            const T *rawZ = reinterpret_cast<const T *>(st + 2 * Ly::RAW_CH) + warp * CPW * TT;
+            const T *rawD = reinterpret_cast<const T *>(st) + warp * rpw * TT;
+            const T *rawU = reinterpret_cast<const T *>(st + Ly::RAW_CH) + warp * rpw * TT;
+            const T *rawZ = reinterpret_cast<const T *>(st + 2 * Ly::RAW_CH) + warp * rpw * TT;
             // (1) Δ and Δ·u, once per element (pairs of steps in f32x2 math)
             const bool full_tile = t0 + TT <= p.L;
 #pragma unroll
