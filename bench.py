@@ -380,6 +380,121 @@ def run_ours(args, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+def run_decode(args, world, rank, local):
+    """One decoding step (ssm_selective_state_update) at the Mamba-2.8B layer
+    width: batch 64 sequences, dim 5120, dstate 16, bf16 io, fp32 state kept
+    on the device.  Memory-bound: reported against the HBM roofline."""
+    import torch
+    import oracle
+    from selective_state_space_50_b200 import ssm_scan
+    from selective_state_space_50_b200.workloads import Workload, generate, to_torch
+
+    w = Workload("decode_step_2p8b", 64, 1, 5120, 16, "bf16", seed=1005 + 7919 * rank,
+                 D_dist="u0.5_1.5")
+    dev = torch.device("cuda", local)
+    inp = generate(w)
+    dv = to_torch(inp, w, dev)
+    sq = {k: (dv[k][..., 0].contiguous() if dv[k] is not None and k in ("u", "delta", "z", "B", "C")
+              else dv[k]) for k in dv}
+    st0 = np.random.default_rng(w.seed).standard_normal((w.batch, w.dim, w.dstate)).astype(np.float32)
+    state = torch.from_numpy(st0).to(dev)
+    out = torch.empty_like(sq["u"])
+    shape = ssm_scan.make_shape(w.batch, w.dim, 1, w.dstate, sq["u"].dtype)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def step():
+        ssm_scan.state_update_raw(shape, state, sq["u"], sq["delta"], sq["A"], sq["B"], sq["C"],
+                                  sq["D"], sq["z"], sq["delta_bias"], True, out, stream)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    with ClockSampler(local) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    t_dev = sum(s.elapsed_time(e) for s, e in zip(starts, ends)) / 1e3
+    t_max = max_over_ranks(t_dev, world)
+    units = w.batch * w.dim * w.dstate
+
+    # end to end: the token's inputs from pinned host memory, the output back;
+    # the state stays on the device (as in a decoding loop)
+    host = {k: sq[k].cpu().pin_memory() for k in ("u", "delta", "z", "B", "C")}
+    dtmp = {k: torch.empty_like(sq[k]) for k in host}
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_h.numel() * out_h.element_size()
+    e2e_steps = max(5, min(args.steps, 50))
+    e_s = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
+    e_e = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
+
+    def e2e_step():
+        for k, t in host.items():
+            dtmp[k].copy_(t, non_blocking=True)
+        o = ssm_scan.selective_state_update(state, dtmp["u"], dtmp["delta"], sq["A"], dtmp["B"],
+                                            dtmp["C"], sq["D"], dtmp["z"], sq["delta_bias"], True,
+                                            out=out)
+        out_h.copy_(o, non_blocking=True)
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    for i in range(e2e_steps):
+        flush.zero_()
+        e_s[i].record(stream)
+        e2e_step()
+        e_e[i].record(stream)
+    torch.cuda.synchronize()
+    t_e2e = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(e_s, e_e)) / 1e3, world)
+    if rank != 0:
+        return
+    peaks, peak_src = measured_peaks()
+    mean_s = t_dev / args.steps
+    es_io = 2
+    alg = (2 * 4 * units + 4 * es_io * w.batch * w.dim + 2 * es_io * w.dstate * w.batch
+           + 4 * w.dim * w.dstate + 8 * w.dim)
+    line = {
+        "metric": "selective-state-update B*D*N elems/s", "value": world * args.steps * units / t_max,
+        "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup),
+        "ms_per_step": t_max / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "dim": w.dim, "dstate": w.dstate,
+                   "io_dtype": w.io_dtype, "state_dtype": "f32",
+                   "parallelism": f"replicas x{world} (independent batches)",
+                   "l2": "flushed between steps (256 MiB write, outside the timed events)"},
+        "roofline": {"bound": "hbm", "achieved": alg / mean_s / 1e9, "peak": float(peaks["hbm_gbs"]),
+                     "unit": "GB/s", "frac": alg / mean_s / 1e9 / float(peaks["hbm_gbs"]),
+                     "traffic": None, "peak_source": peak_src, "alg_bytes": alg},
+        "clocks": clk.summary(),
+        "e2e": {"value": world * e2e_steps * units / t_e2e, "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        st64 = st0.astype(np.float64)
+        t0 = time.perf_counter()
+        n = 0
+        while time.perf_counter() - t0 < min(args.cpu_budget, 5.0) or n == 0:
+            oracle.step(st64, inp["u_f64"][..., 0], inp["delta_f64"][..., 0], inp["A_f64"],
+                        inp["B_f64"][..., 0], inp["C_f64"][..., 0], inp["D_f64"], inp["z_f64"][..., 0],
+                        inp["delta_bias_f64"], True)
+            n += 1
+        el = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": n * units / el, "unit": UNIT, "cores": oracle.max_threads(),
+                                "kind": "oracle",
+                                "sample": f"{n} full steps of {w.name} (fp64), {el:.1f} s"}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -392,11 +507,15 @@ def main():
                     help="workload to time (default: the Mamba-130M layer shape)")
     ap.add_argument("--seqlen", type=int, default=0,
                     help="override the workload's sequence length (for profiling small cases)")
+    ap.add_argument("--decode", action="store_true",
+                    help="time the single-step recurrent update instead of the scan")
     args = ap.parse_args()
     world, rank, local = dist_setup(args)
     try:
         if args.impl == "reference":
             run_reference(args, world, rank)
+        elif args.decode:
+            run_decode(args, world, rank, local)
         else:
             run_ours(args, world, rank, local)
     finally:

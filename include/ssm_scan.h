@@ -190,6 +190,35 @@ ssm_status_t ssm_selective_scan_bwd_noalloc(const ssm_shape_t *shape,
                                             float *ddelta_bias, void *stream);
 
 /*
+ * One step of the recurrence for decoding (the recurrent form of the
+ * selective SSM: 정보관리기술사 학습 노트, "상태공간 모델(SSM)과 Mamba 아키텍처"
+ * §2, with the selective Δ, B, C of booiljung.github.io §1.1).  For each
+ * (b, d), in place:
+ *   Δ = softplus(delta[b][d] + delta_bias[d])   (raw sum if delta_softplus == 0)
+ *   state[b][d][n] = exp(Δ A[d][n]) state[b][d][n] + Δ B[b][n] u[b][d]
+ *   y = Σ_n C[b][n] state[b][d][n] + D[d] u[b][d];  out[b][d] = y z σ(z)
+ * This equals ssm_selective_scan_fwd over one step started from `state`.
+ *
+ *  shape        : seqlen must be 1; u, delta, z, out are [batch][dim] and
+ *                 B, C are [batch][dstate], all in the io dtype.
+ *  state        : [batch][dim][dstate] fp32, read and overwritten (caller
+ *                 owned); 16-byte alignment of state and A enables vector
+ *                 access but is not required.
+ *  A, D, delta_bias, z : as in ssm_selective_scan_fwd (D, z, delta_bias
+ *                 optional).
+ *  out          : required, io dtype; may not alias the state or an input.
+ * Asynchronous on `stream`; no device allocation.
+ * Errors: SSM_ERR_INVALID_ARG (seqlen != 1, NULL or misaligned pointers,
+ * host pointers, aliasing), SSM_ERR_UNSUPPORTED (dstate), SSM_ERR_CUDA.
+ */
+ssm_status_t ssm_selective_state_update(const ssm_shape_t *shape, float *state,
+                                        const void *u, const void *delta,
+                                        const float *A, const void *B, const void *C,
+                                        const float *D, const void *z,
+                                        const float *delta_bias, int delta_softplus,
+                                        void *out, void *stream);
+
+/*
  * Synchronises `stream`, then reports (and clears) the device-side error word
  * that kernels set when one of their bounded waits gives up: SSM_OK if none
  * did since the previous call, SSM_ERR_TIMEOUT otherwise.  Kernel waits are

@@ -262,6 +262,40 @@ ssm_status_t ssm_selective_scan_bwd(const ssm_shape_t *shape, const void *u, con
     return ok();
 }
 
+ssm_status_t ssm_selective_state_update(const ssm_shape_t *shape, float *state, const void *u,
+                                        const void *delta, const float *A, const void *B,
+                                        const void *C, const float *D, const void *z,
+                                        const float *delta_bias, int delta_softplus, void *out,
+                                        void *stream) {
+    SSM_TRY(check_shape(shape));
+    if (shape->seqlen != 1)
+        return fail(SSM_ERR_INVALID_ARG, "a single step needs seqlen == 1 (got %d)", shape->seqlen);
+    const size_t es = esize(shape->io_dtype);
+    SSM_TRY(check_ptr(state, "state", 4, true));
+    SSM_TRY(check_ptr(u, "u", es, true));
+    SSM_TRY(check_ptr(delta, "delta", es, true));
+    SSM_TRY(check_ptr(A, "A", 4, true));
+    SSM_TRY(check_ptr(B, "B", es, true));
+    SSM_TRY(check_ptr(C, "C", es, true));
+    SSM_TRY(check_ptr(D, "D", 4, false));
+    SSM_TRY(check_ptr(z, "z", es, false));
+    SSM_TRY(check_ptr(delta_bias, "delta_bias", 4, false));
+    SSM_TRY(check_ptr(out, "out", es, true));
+    const void *ins[] = {state, u, delta, A, B, C, D, z, delta_bias};
+    for (const void *q : ins)
+        if (out == q) return fail(SSM_ERR_INVALID_ARG, "out may not alias an input or the state");
+    ssm::StepParams p{};
+    p.state = state; p.u = u; p.delta = delta; p.A = A; p.B = B; p.C = C; p.D = D; p.z = z;
+    p.delta_bias = delta_bias; p.out = out;
+    p.P = (long long)shape->batch * shape->dim; p.dim = shape->dim; p.N = shape->dstate;
+    p.softplus = delta_softplus != 0;
+    p.io_bf16 = shape->io_dtype == SSM_BF16;
+    p.vec_ok = aligned16(state) && aligned16(A);
+    cudaError_t e = ssm::launch_state_update(p, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "ssm_selective_state_update launch");
+    return ok();
+}
+
 ssm_status_t ssm_device_error_status(void *stream) {
     int v = 0;
     cudaError_t e = ssm::read_and_clear_device_error(&v, static_cast<cudaStream_t>(stream));

@@ -40,6 +40,25 @@ struct BwdParams {
     bool vec_ok;
 };
 
+struct StepParams {
+    float *state;                  // [batch][dim][N], updated in place
+    const void *u, *delta;         // [batch][dim]
+    const float *A;                // [dim][N]
+    const void *B, *C;             // [batch][N]
+    const float *D;
+    const void *z;
+    const float *delta_bias;
+    void *out;                     // [batch][dim]
+    long long P;                   // batch * dim
+    int dim, N;
+    int softplus;
+    bool io_bf16;
+    bool vec_ok;                   // state and A 16-byte aligned (vector access)
+};
+
+// Single-step recurrent update (ssm_step.cu).
+cudaError_t launch_state_update(const StepParams &p, cudaStream_t stream);
+
 enum class FwdKernel { kAuto = 0, kGeneral = 1, kTma = 2 };
 FwdKernel fwd_kernel_choice();
 

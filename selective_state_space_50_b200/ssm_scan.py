@@ -25,7 +25,7 @@ CKPT_CHUNK = 8  # SSM_CKPT_CHUNK in include/ssm_scan.h
 EXPORTS = ("ssm_version", "ssm_last_error_string", "ssm_selective_scan_ckpt_bytes",
            "ssm_selective_scan_fwd", "ssm_selective_scan_bwd_scratch_bytes",
            "ssm_selective_scan_bwd", "ssm_device_error_status",
-           "ssm_selective_scan_bwd_noalloc")
+           "ssm_selective_scan_bwd_noalloc", "ssm_selective_state_update")
 NOALLOC_SCRATCH_BYTES = 32 << 20  # SSM_NOALLOC_SCRATCH_BYTES in include/ssm_scan.h
 
 
@@ -68,6 +68,8 @@ def load_library(path: str = LIB_PATH):
     lib.ssm_device_error_status.restype = i
     lib.ssm_selective_scan_bwd_noalloc.argtypes = [sp] + [vp] * 8 + [i] + [vp] * 10
     lib.ssm_selective_scan_bwd_noalloc.restype = i
+    lib.ssm_selective_state_update.argtypes = [sp] + [vp] * 9 + [i] + [vp] * 2
+    lib.ssm_selective_state_update.restype = i
     _lib = lib
     return lib
 
@@ -151,6 +153,15 @@ def bwd_noalloc_raw(shape: Shape, u, delta, A, B, C, D, z, delta_bias, delta_sof
         _ptr(dB), _ptr(dC), _ptr(dD), _ptr(dz), _ptr(ddelta_bias), _stream_ptr(stream)))
 
 
+def state_update_raw(shape: Shape, state, u, delta, A, B, C, D, z, delta_bias,
+                     delta_softplus: bool, out, stream=None):
+    """Direct call of ssm_selective_state_update (one decoding step, state
+    updated in place)."""
+    _check(load_library().ssm_selective_state_update(
+        ctypes.byref(shape), _ptr(state), _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+        _ptr(z), _ptr(delta_bias), int(bool(delta_softplus)), _ptr(out), _stream_ptr(stream)))
+
+
 def _need(t, name, dtype=None, cuda=True):
     if t is None:
         return
@@ -182,6 +193,26 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None,
           if return_ckpt else None)
     fwd_raw(shape, u, delta, A, B, C, D, z, delta_bias, delta_softplus, out, last, ck, stream)
     return out, last, ck
+
+
+def selective_state_update(state, u, delta, A, B, C, D=None, z=None, delta_bias=None,
+                           delta_softplus: bool = True, out=None, stream=None):
+    """One decoding step: advances `state` ([batch, dim, dstate] float32) in
+    place by one token and returns out [batch, dim].  u, delta, z are
+    [batch, dim] and B, C [batch, dstate] in one io dtype; A, D, delta_bias
+    are float32."""
+    io = u.dtype
+    for t, n in ((u, "u"), (delta, "delta"), (B, "B"), (C, "C"), (z, "z")):
+        _need(t, n, io)
+    for t, n in ((state, "state"), (A, "A"), (D, "D"), (delta_bias, "delta_bias")):
+        _need(t, n, torch.float32)
+    if u.dim() != 2 or state.dim() != 3 or tuple(state.shape) != (u.shape[0], u.shape[1], A.shape[1]):
+        raise ValueError("u must be [batch, dim], A [dim, dstate] and state [batch, dim, dstate]")
+    shape = make_shape(u.shape[0], u.shape[1], 1, A.shape[1], io)
+    if out is None:
+        out = torch.empty_like(u)
+    state_update_raw(shape, state, u, delta, A, B, C, D, z, delta_bias, delta_softplus, out, stream)
+    return out
 
 
 def selective_scan_bwd(u, delta, A, B, C, D, z, delta_bias, delta_softplus: bool, dout,

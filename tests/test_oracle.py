@@ -229,6 +229,36 @@ def _combine(later, earlier):
     return Aj * Ai, Aj * bi + bj
 
 
+def test_step_hand_computed_two_states():
+    """One decoding step from a nonzero state, written out by hand: N=2,
+    softplus on, gate on (h' = exp(Δa) h + Δ B u, y = C·h' + D u, y z σ(z))."""
+    h = np.array([[[0.3, -1.2]]])
+    a = np.array([[-0.7, -2.0]])
+    Bv, Cv = np.array([[1.5, -0.25]]), np.array([[-1.0, 2.0]])
+    x, r, zz, Dd, bias = 0.8, -0.4, 1.3, 0.6, 0.1
+    dt = math.log1p(math.exp(r + bias))
+    h_new = [math.exp(dt * a[0, n]) * h[0, 0, n] + dt * Bv[0, n] * x for n in range(2)]
+    y = Cv[0, 0] * h_new[0] + Cv[0, 1] * h_new[1] + Dd * x
+    want = y * zz / (1.0 + math.exp(-zz))
+    out, st = oracle.step(h, np.array([[x]]), np.array([[r]]), a, Bv, Cv, D=np.array([Dd]),
+                          z=np.array([[zz]]), delta_bias=np.array([bias]))
+    assert abs(out[0, 0] - want) < 1e-14
+    np.testing.assert_allclose(st[0, 0], h_new, rtol=1e-14, atol=1e-15)
+
+
+def test_steps_reproduce_the_scan():
+    """L single steps started from zero give the scan's outputs and final state."""
+    c = rand_case(21, batch=2, dim=3, L=9, N=4)
+    out, last = oracle.fwd(c["u"], c["delta"], c["A"], c["B"], c["C"], c["D"], c["z"],
+                           c["delta_bias"], True)
+    st = np.zeros((2, 3, 4))
+    for t in range(9):
+        y, st = oracle.step(st, c["u"][..., t], c["delta"][..., t], c["A"], c["B"][..., t],
+                            c["C"][..., t], c["D"], c["z"][..., t], c["delta_bias"], True)
+        np.testing.assert_allclose(y, out[..., t], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(st, last, rtol=1e-12, atol=1e-13)
+
+
 def test_combine_operator_is_associative():
     r = rng(9)
     for _ in range(100):
