@@ -202,14 +202,15 @@ ssm_status_t ssm_selective_scan_bwd_noalloc(const ssm_shape_t *shape,
  *  shape        : seqlen must be 1; u, delta, z, out are [batch][dim] and
  *                 B, C are [batch][dstate], all in the io dtype.
  *  state        : [batch][dim][dstate] fp32, read and overwritten (caller
- *                 owned); 16-byte alignment of state and A enables vector
- *                 access but is not required.
+ *                 owned); 16-byte alignment of state, A, B and C enables
+ *                 vector access but is not required.
  *  A, D, delta_bias, z : as in ssm_selective_scan_fwd (D, z, delta_bias
  *                 optional).
  *  out          : required, io dtype; may not alias the state or an input.
  * Asynchronous on `stream`; no device allocation.
  * Errors: SSM_ERR_INVALID_ARG (seqlen != 1, NULL or misaligned pointers,
- * host pointers, aliasing), SSM_ERR_UNSUPPORTED (dstate), SSM_ERR_CUDA.
+ * host pointers, aliasing), SSM_ERR_UNSUPPORTED (dstate, batch > 65535),
+ * SSM_ERR_CUDA.
  */
 ssm_status_t ssm_selective_state_update(const ssm_shape_t *shape, float *state,
                                         const void *u, const void *delta,

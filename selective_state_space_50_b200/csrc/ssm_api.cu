@@ -270,6 +270,8 @@ ssm_status_t ssm_selective_state_update(const ssm_shape_t *shape, float *state, 
     SSM_TRY(check_shape(shape));
     if (shape->seqlen != 1)
         return fail(SSM_ERR_INVALID_ARG, "a single step needs seqlen == 1 (got %d)", shape->seqlen);
+    if (shape->batch > 65535)
+        return fail(SSM_ERR_UNSUPPORTED, "batch %d > 65535 for a single step", shape->batch);
     const size_t es = esize(shape->io_dtype);
     SSM_TRY(check_ptr(state, "state", 4, true));
     SSM_TRY(check_ptr(u, "u", es, true));
@@ -290,7 +292,7 @@ ssm_status_t ssm_selective_state_update(const ssm_shape_t *shape, float *state, 
     p.P = (long long)shape->batch * shape->dim; p.dim = shape->dim; p.N = shape->dstate;
     p.softplus = delta_softplus != 0;
     p.io_bf16 = shape->io_dtype == SSM_BF16;
-    p.vec_ok = aligned16(state) && aligned16(A);
+    p.vec_ok = aligned16(state) && aligned16(A) && aligned16(B) && aligned16(C);
     cudaError_t e = ssm::launch_state_update(p, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "ssm_selective_state_update launch");
     return ok();

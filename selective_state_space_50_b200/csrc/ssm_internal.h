@@ -53,7 +53,7 @@ struct StepParams {
     int dim, N;
     int softplus;
     bool io_bf16;
-    bool vec_ok;                   // state and A 16-byte aligned (vector access)
+    bool vec_ok;                   // state, A, B, C 16-byte aligned (vector access)
 };
 
 // Single-step recurrent update (ssm_step.cu).

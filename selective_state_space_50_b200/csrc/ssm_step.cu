@@ -20,42 +20,68 @@ namespace ssm {
 
 namespace {
 
-template <typename T, int SPT>
+// States per thread (at most; a multiple of 4 for vector access).
+#ifndef SSM_STEP_SPT
+#define SSM_STEP_SPT 4
+#endif
+constexpr int kStepSpt = SSM_STEP_SPT;
+
+template <typename T, int SPT, bool VEC>
 __device__ __forceinline__ void load_io(const T *p, float (&f)[SPT]) {
+    if constexpr (VEC && SPT % 4 == 0 && sizeof(T) == 2) {
 #pragma unroll
-    for (int i = 0; i < SPT; ++i) f[i] = IO<T>::to_f(p[i]);
+        for (int i = 0; i < SPT; i += 4) {
+            const uint2 q = *reinterpret_cast<const uint2 *>(p + i);
+            f[i] = __uint_as_float(q.x << 16); f[i + 1] = __uint_as_float(q.x & 0xffff0000u);
+            f[i + 2] = __uint_as_float(q.y << 16); f[i + 3] = __uint_as_float(q.y & 0xffff0000u);
+        }
+    } else if constexpr (VEC && SPT % 4 == 0 && sizeof(T) == 4) {
+#pragma unroll
+        for (int i = 0; i < SPT; i += 4) {
+            const float4 q = *reinterpret_cast<const float4 *>(p + i);
+            f[i] = q.x; f[i + 1] = q.y; f[i + 2] = q.z; f[i + 3] = q.w;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < SPT; ++i) f[i] = IO<T>::to_f(p[i]);
+    }
 }
 
 template <typename T, int N, bool VEC>
 __global__ void __launch_bounds__(256) state_update_kernel(const StepParams p) {
-    constexpr int SPT = N < 4 ? N : 4;     // states per thread
-    constexpr int TPC = N / SPT;           // threads per channel (a power of two, <= 8)
-    const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    const long long ch_raw = gid / TPC;
-    const int q = (int)(gid % TPC);
-    const bool ok = ch_raw < p.P;
-    const long long ch = ok ? ch_raw : p.P - 1;   // out-of-range threads mirror the last channel
-    const int b = (int)(ch / p.dim), d = (int)(ch % p.dim);
+    constexpr int SPT = N < kStepSpt ? N : kStepSpt;   // states per thread
+    constexpr int TPC = N / SPT;           // threads per channel (a power of two)
+    // grid: x covers the channels of one batch row, y is the batch row
+    const unsigned b = blockIdx.y;
+    const unsigned t = blockIdx.x * blockDim.x + threadIdx.x;
+    const unsigned dim = (unsigned)p.dim;
+    const unsigned d_raw = t / TPC;
+    const int q = (int)(t % TPC);
+    const bool ok = d_raw < dim;
+    const unsigned d = ok ? d_raw : dim - 1;   // out-of-range groups mirror the last channel
+    const unsigned ch = b * dim + d;
 
     float h[SPT], a2[SPT], bb[SPT], cc[SPT];
-    float *st = p.state + ch * N + q * SPT;
+    float *st = p.state + (size_t)ch * N + q * SPT;   // batch * dim * N may exceed 2^32
     const float *ar = p.A + (size_t)d * N + q * SPT;
-    if constexpr (VEC && SPT == 4) {
-        const float4 hv = *reinterpret_cast<const float4 *>(st);
-        const float4 av = __ldg(reinterpret_cast<const float4 *>(ar));
-        h[0] = hv.x; h[1] = hv.y; h[2] = hv.z; h[3] = hv.w;
-        a2[0] = av.x; a2[1] = av.y; a2[2] = av.z; a2[3] = av.w;
+    if constexpr (VEC && SPT % 4 == 0) {
+#pragma unroll
+        for (int i = 0; i < SPT; i += 4) {
+            const float4 hv = *reinterpret_cast<const float4 *>(st + i);
+            const float4 av = __ldg(reinterpret_cast<const float4 *>(ar + i));
+            h[i] = hv.x; h[i + 1] = hv.y; h[i + 2] = hv.z; h[i + 3] = hv.w;
+            a2[i] = av.x; a2[i + 1] = av.y; a2[i + 2] = av.z; a2[i + 3] = av.w;
+        }
     } else {
 #pragma unroll
         for (int i = 0; i < SPT; ++i) { h[i] = st[i]; a2[i] = __ldg(ar + i); }
     }
-    const T *Bp = static_cast<const T *>(p.B) + (size_t)b * N + q * SPT;
-    const T *Cp = static_cast<const T *>(p.C) + (size_t)b * N + q * SPT;
-    load_io<T, SPT>(Bp, bb);
-    load_io<T, SPT>(Cp, cc);
-
+    load_io<T, SPT, VEC>(static_cast<const T *>(p.B) + b * N + q * SPT, bb);
+    load_io<T, SPT, VEC>(static_cast<const T *>(p.C) + b * N + q * SPT, cc);
     const float u = IO<T>::to_f(static_cast<const T *>(p.u)[ch]);
     const float r = IO<T>::to_f(static_cast<const T *>(p.delta)[ch]) + (p.delta_bias ? p.delta_bias[d] : 0.f);
+    const float zz = p.z ? IO<T>::to_f(static_cast<const T *>(p.z)[ch]) : 0.f;
+
     const float dt = p.softplus ? softplus_fast(r) : r;
     const float du = dt * u;
     float y = 0.f;
@@ -68,32 +94,32 @@ __global__ void __launch_bounds__(256) state_update_kernel(const StepParams p) {
 #pragma unroll
     for (int m = TPC / 2; m >= 1; m >>= 1) y += __shfl_xor_sync(0xffffffffu, y, m);
     if (!ok) return;
-    if constexpr (VEC && SPT == 4) {
-        *reinterpret_cast<float4 *>(st) = make_float4(h[0], h[1], h[2], h[3]);
+    if constexpr (VEC && SPT % 4 == 0) {
+#pragma unroll
+        for (int i = 0; i < SPT; i += 4)
+            *reinterpret_cast<float4 *>(st + i) = make_float4(h[i], h[i + 1], h[i + 2], h[i + 3]);
     } else {
 #pragma unroll
         for (int i = 0; i < SPT; ++i) st[i] = h[i];
     }
     if (q == 0) {
         y = fmaf(p.D ? p.D[d] : 0.f, u, y);
-        if (p.z) {
-            const float z = IO<T>::to_f(static_cast<const T *>(p.z)[ch]);
-            y *= z * sigmoid(z);
-        }
+        if (p.z) y *= zz * sigmoid(zz);
         static_cast<T *>(p.out)[ch] = IO<T>::from_f(y);
     }
 }
 
 template <typename T, int N>
 cudaError_t launch_step_n(const StepParams &p, cudaStream_t stream) {
-    constexpr int SPT = N < 4 ? N : 4;
+    constexpr int SPT = N < kStepSpt ? N : kStepSpt;
     constexpr int TPC = N / SPT;
-    const long long threads = p.P * TPC;
     const int block = 256;
-    const long long grid = (threads + block - 1) / block;
-    if (grid > 0x7fffffffLL) return cudaErrorInvalidValue;
-    if (p.vec_ok) state_update_kernel<T, N, true><<<(unsigned)grid, block, 0, stream>>>(p);
-    else state_update_kernel<T, N, false><<<(unsigned)grid, block, 0, stream>>>(p);
+    const long long gx = ((long long)p.dim * TPC + block - 1) / block;
+    const long long batch = p.P / p.dim;
+    if (gx > 0x7fffffffLL || batch > 65535) return cudaErrorInvalidValue;
+    const dim3 grid((unsigned)gx, (unsigned)batch);
+    if (p.vec_ok) state_update_kernel<T, N, true><<<grid, block, 0, stream>>>(p);
+    else state_update_kernel<T, N, false><<<grid, block, 0, stream>>>(p);
     return cudaGetLastError();
 }
 
