@@ -47,65 +47,86 @@ __device__ __forceinline__ void load_io(const T *p, float (&f)[SPT]) {
     }
 }
 
+// Channels per thread: all loads of the CPT channels are issued before any
+// arithmetic, so that more memory requests are in flight per thread.
+#ifndef SSM_STEP_CPT
+#define SSM_STEP_CPT 2
+#endif
+constexpr int kStepCpt = SSM_STEP_CPT;
+
 template <typename T, int N, bool VEC>
 __global__ void __launch_bounds__(256) state_update_kernel(const StepParams p) {
     constexpr int SPT = N < kStepSpt ? N : kStepSpt;   // states per thread
     constexpr int TPC = N / SPT;           // threads per channel (a power of two)
-    // grid: x covers the channels of one batch row, y is the batch row
+    constexpr int CPT = kStepCpt;
+    // grid: x covers the channels of one batch row (CPT per thread group,
+    // strided by the x extent), y is the batch row
     const unsigned b = blockIdx.y;
     const unsigned t = blockIdx.x * blockDim.x + threadIdx.x;
+    const unsigned stride = gridDim.x * blockDim.x / TPC;
     const unsigned dim = (unsigned)p.dim;
-    const unsigned d_raw = t / TPC;
     const int q = (int)(t % TPC);
-    const bool ok = d_raw < dim;
-    const unsigned d = ok ? d_raw : dim - 1;   // out-of-range groups mirror the last channel
-    const unsigned ch = b * dim + d;
 
-    float h[SPT], a2[SPT], bb[SPT], cc[SPT];
-    float *st = p.state + (size_t)ch * N + q * SPT;   // batch * dim * N may exceed 2^32
-    const float *ar = p.A + (size_t)d * N + q * SPT;
-    if constexpr (VEC && SPT % 4 == 0) {
-#pragma unroll
-        for (int i = 0; i < SPT; i += 4) {
-            const float4 hv = *reinterpret_cast<const float4 *>(st + i);
-            const float4 av = __ldg(reinterpret_cast<const float4 *>(ar + i));
-            h[i] = hv.x; h[i + 1] = hv.y; h[i + 2] = hv.z; h[i + 3] = hv.w;
-            a2[i] = av.x; a2[i + 1] = av.y; a2[i + 2] = av.z; a2[i + 3] = av.w;
-        }
-    } else {
-#pragma unroll
-        for (int i = 0; i < SPT; ++i) { h[i] = st[i]; a2[i] = __ldg(ar + i); }
-    }
+    float h[CPT][SPT], a2[CPT][SPT], bb[SPT], cc[SPT];
+    float u[CPT], r[CPT], zz[CPT];
+    unsigned ds[CPT];
+    bool oks[CPT];
     load_io<T, SPT, VEC>(static_cast<const T *>(p.B) + b * N + q * SPT, bb);
     load_io<T, SPT, VEC>(static_cast<const T *>(p.C) + b * N + q * SPT, cc);
-    const float u = IO<T>::to_f(static_cast<const T *>(p.u)[ch]);
-    const float r = IO<T>::to_f(static_cast<const T *>(p.delta)[ch]) + (p.delta_bias ? p.delta_bias[d] : 0.f);
-    const float zz = p.z ? IO<T>::to_f(static_cast<const T *>(p.z)[ch]) : 0.f;
-
-    const float dt = p.softplus ? softplus_fast(r) : r;
-    const float du = dt * u;
-    float y = 0.f;
 #pragma unroll
-    for (int i = 0; i < SPT; ++i) {
-        const float a = ex2(dt * (a2[i] * SSM_LOG2E));
-        h[i] = fmaf(a, h[i], du * bb[i]);
-        y = fmaf(cc[i], h[i], y);
+    for (int k = 0; k < CPT; ++k) {
+        const unsigned d_raw = t / TPC + k * stride;
+        oks[k] = d_raw < dim;
+        const unsigned d = oks[k] ? d_raw : dim - 1;   // out-of-range groups mirror the last channel
+        ds[k] = d;
+        const unsigned ch = b * dim + d;
+        const float *st = p.state + (size_t)ch * N + q * SPT;   // batch * dim * N may exceed 2^32
+        const float *ar = p.A + (size_t)d * N + q * SPT;
+        if constexpr (VEC && SPT % 4 == 0) {
+#pragma unroll
+            for (int i = 0; i < SPT; i += 4) {
+                const float4 hv = *reinterpret_cast<const float4 *>(st + i);
+                const float4 av = __ldg(reinterpret_cast<const float4 *>(ar + i));
+                h[k][i] = hv.x; h[k][i + 1] = hv.y; h[k][i + 2] = hv.z; h[k][i + 3] = hv.w;
+                a2[k][i] = av.x; a2[k][i + 1] = av.y; a2[k][i + 2] = av.z; a2[k][i + 3] = av.w;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < SPT; ++i) { h[k][i] = st[i]; a2[k][i] = __ldg(ar + i); }
+        }
+        u[k] = IO<T>::to_f(static_cast<const T *>(p.u)[ch]);
+        r[k] = IO<T>::to_f(static_cast<const T *>(p.delta)[ch]) + (p.delta_bias ? p.delta_bias[d] : 0.f);
+        zz[k] = p.z ? IO<T>::to_f(static_cast<const T *>(p.z)[ch]) : 0.f;
     }
 #pragma unroll
-    for (int m = TPC / 2; m >= 1; m >>= 1) y += __shfl_xor_sync(0xffffffffu, y, m);
-    if (!ok) return;
-    if constexpr (VEC && SPT % 4 == 0) {
+    for (int k = 0; k < CPT; ++k) {
+        const float dt = p.softplus ? softplus_fast(r[k]) : r[k];
+        const float du = dt * u[k];
+        float y = 0.f;
 #pragma unroll
-        for (int i = 0; i < SPT; i += 4)
-            *reinterpret_cast<float4 *>(st + i) = make_float4(h[i], h[i + 1], h[i + 2], h[i + 3]);
-    } else {
+        for (int i = 0; i < SPT; ++i) {
+            const float a = ex2(dt * (a2[k][i] * SSM_LOG2E));
+            h[k][i] = fmaf(a, h[k][i], du * bb[i]);
+            y = fmaf(cc[i], h[k][i], y);
+        }
 #pragma unroll
-        for (int i = 0; i < SPT; ++i) st[i] = h[i];
-    }
-    if (q == 0) {
-        y = fmaf(p.D ? p.D[d] : 0.f, u, y);
-        if (p.z) y *= zz * sigmoid(zz);
-        static_cast<T *>(p.out)[ch] = IO<T>::from_f(y);
+        for (int m = TPC / 2; m >= 1; m >>= 1) y += __shfl_xor_sync(0xffffffffu, y, m);
+        if (!oks[k]) continue;
+        const unsigned ch = b * dim + ds[k];
+        float *st = p.state + (size_t)ch * N + q * SPT;
+        if constexpr (VEC && SPT % 4 == 0) {
+#pragma unroll
+            for (int i = 0; i < SPT; i += 4)
+                *reinterpret_cast<float4 *>(st + i) = make_float4(h[k][i], h[k][i + 1], h[k][i + 2], h[k][i + 3]);
+        } else {
+#pragma unroll
+            for (int i = 0; i < SPT; ++i) st[i] = h[k][i];
+        }
+        if (q == 0) {
+            y = fmaf(p.D ? p.D[ds[k]] : 0.f, u[k], y);
+            if (p.z) y *= zz[k] * sigmoid(zz[k]);
+            static_cast<T *>(p.out)[ch] = IO<T>::from_f(y);
+        }
     }
 }
 
@@ -114,7 +135,8 @@ cudaError_t launch_step_n(const StepParams &p, cudaStream_t stream) {
     constexpr int SPT = N < kStepSpt ? N : kStepSpt;
     constexpr int TPC = N / SPT;
     const int block = 256;
-    const long long gx = ((long long)p.dim * TPC + block - 1) / block;
+    const long long groups = ((long long)p.dim + kStepCpt - 1) / kStepCpt;
+    const long long gx = (groups * TPC + block - 1) / block;
     const long long batch = p.P / p.dim;
     if (gx > 0x7fffffffLL || batch > 65535) return cudaErrorInvalidValue;
     const dim3 grid((unsigned)gx, (unsigned)batch);
