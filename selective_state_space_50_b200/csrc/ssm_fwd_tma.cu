@@ -143,7 +143,9 @@ __device__ __forceinline__ void load_pairs8_at<float>(const float *lo, const flo
     v[2] = make_float2(b.x, b.y); v[3] = make_float2(b.z, b.w);
 }
 
-template <typename T, int NT, int NS, int TT, int NWC, int STAGES>
+// FL < 0: the gate, softplus and checkpoint options are read at run time;
+// otherwise they are compile-time bits (1: gate z, 2: softplus, 4: checkpoints).
+template <typename T, int NT, int NS, int TT, int NWC, int STAGES, int FL>
 __global__ void __launch_bounds__((NWC + 1) * 32, 1)
 fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constant__ CUtensorMap m_u,
                const __grid_constant__ CUtensorMap m_z, const __grid_constant__ CUtensorMap m_B,
@@ -152,6 +154,9 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
     constexpr int N = Ly::N, CPW = Ly::CPW, WS = Ly::WS, CHUNK = Ly::CHUNK;
     constexpr int IPL = Ly::ITEMS / 32;   // prep/epilogue items per lane
     constexpr int CPR = TT / CHUNK;       // chunks per row
+    const bool has_z = FL < 0 ? p.has_z != 0 : (FL & 1) != 0;
+    const bool softplus = FL < 0 ? p.softplus != 0 : (FL & 2) != 0;
+    float *const ckpt = (FL < 0 || (FL & 4)) ? p.ckpt : nullptr;
 
     extern __shared__ __align__(128) uint8_t smem_raw[];
     // 1024-byte aligned base: the 128B-swizzle pattern of the B/C tiles repeats
@@ -189,7 +194,7 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
         if (lane != 0) return;
         prefetch_tensormap(&m_delta);
         prefetch_tensormap(&m_u);
-        if (p.has_z) prefetch_tensormap(&m_z);
+        if (has_z) prefetch_tensormap(&m_z);
         prefetch_tensormap(&m_B);
         prefetch_tensormap(&m_C);
         int issued = 0;
@@ -207,12 +212,12 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
             }
             const int t0 = tile * TT;
             uint8_t *st = smem + s * Ly::STAGE;
-            const uint32_t bytes = (uint32_t)(p.rows_max * Ly::RAW_ROW * (2 + p.has_z) +
+            const uint32_t bytes = (uint32_t)(p.rows_max * Ly::RAW_ROW * (has_z ? 3 : 2) +
                                               2 * nb * N * Ly::RAW_ROW);
             mbar_arrive_expect_tx(full + s, bytes);
             tma_load_2d(st, &m_delta, t0, q0, full + s);
             tma_load_2d(st + Ly::RAW_CH, &m_u, t0, q0, full + s);
-            if (p.has_z) tma_load_2d(st + 2 * Ly::RAW_CH, &m_z, t0, q0, full + s);
+            if (has_z) tma_load_2d(st + 2 * Ly::RAW_CH, &m_z, t0, q0, full + s);
             for (int bs = 0; bs < nb; ++bs)
                 for (int pc = 0; pc < Ly::NPIECE; ++pc) {
                     const int off = Ly::kBC0 + pc * Ly::PIECE + bs * N * Ly::PW;
@@ -307,7 +312,7 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
 #pragma unroll
                     for (int k = 0; k < V; k += 2) {
                         const float2 r = __fadd2_rn(make_float2(dr[k], dr[k + 1]), make_float2(bias[i], bias[i]));
-                        float2 d2 = p.softplus ? softplus_fast2(r) : r;
+                        float2 d2 = softplus ? softplus_fast2(r) : r;
                         if (!full_tile) {
                             const bool ok0 = irow[i] >= 0 && (t0 + t + v0 + k) < p.L;
                             const bool ok1 = irow[i] >= 0 && (t0 + t + v0 + k + 1) < p.L;
@@ -343,7 +348,7 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
             };
             const int rr0 = bsel * N + g * NS;
             float *myY = wY + (g * CPW + c) * WS;
-            float *ck_row = (live && p.ckpt) ? p.ckpt + (size_t)(wrow0 + c) * p.n_ckpt * N + g * NS : nullptr;
+            float *ck_row = (live && ckpt) ? ckpt + (size_t)(wrow0 + c) * p.n_ckpt * N + g * NS : nullptr;
             static_assert(SSM_CKPT_CHUNK == 8, "checkpoints are written per 8-step block");
             // one 8-step block of the recurrence; USE_POLY evaluates some of the
             // exponentials with ex2_poly2 on the FMA pipe instead of the SFU
@@ -432,12 +437,12 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                     constexpr int V = IO<T>::kVec;
                     float uu[V], zz[V], o[V];
                     IO<T>::unpack(*reinterpret_cast<const uint4 *>(rawU + rl * TT + t + v0), uu);
-                    if (p.has_z) IO<T>::unpack(*reinterpret_cast<const uint4 *>(rawZ + rl * TT + t + v0), zz);
+                    if (has_z) IO<T>::unpack(*reinterpret_cast<const uint4 *>(rawZ + rl * TT + t + v0), zz);
 #pragma unroll
                     for (int k = 0; k < V; k += 2) {
                         float2 yy = __ffma2_rn(make_float2(Dd[i], Dd[i]), make_float2(uu[k], uu[k + 1]),
                                                make_float2(y[v0 + k], y[v0 + k + 1]));
-                        if (p.has_z) {
+                        if (has_z) {
                             if constexpr (sizeof(T) == 2) {
                                 yy = __fmul2_rn(yy, silu_tanh2(make_float2(zz[k], zz[k + 1])));
                             } else {
@@ -461,7 +466,7 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
 // ------------------------------------------------------------------ host side
 
 
-template <typename T, int NT, int NS, int TT, int NWC, int STAGES>
+template <typename T, int NT, int NS, int TT, int NWC, int STAGES, int FL>
 cudaError_t launch_cfg(const FwdParams &fp, cudaStream_t stream) {
     using Ly = TmaLayout<T, NT, NS, TT, NWC, STAGES>;
     const int P = fp.batch * fp.dim;
@@ -484,7 +489,7 @@ cudaError_t launch_cfg(const FwdParams &fp, cudaStream_t stream) {
     p.softplus = fp.softplus; p.has_z = fp.z != nullptr; p.rows_max = rows_max;
     p.err = device_error_word();
     if (!p.err) return cudaErrorInvalidDevice;
-    auto kern = fwd_tma_kernel<T, NT, NS, TT, NWC, STAGES>;
+    auto kern = fwd_tma_kernel<T, NT, NS, TT, NWC, STAGES, FL>;
     static bool attr_done = false;
     if (!attr_done) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Ly::kAlloc);
@@ -533,7 +538,14 @@ SSM_TMA_CFG(float, 8, 8, 8, 2)
 template <typename T, int N, int NT>
 cudaError_t launch_nt(const FwdParams &fp, cudaStream_t stream) {
     using C = TmaCfg<T, N, NT>;
-    return launch_cfg<T, NT, N / NT, C::TT, C::NWC, C::STAGES>(fp, stream);
+    // the benchmarked bf16 dstate-16 splits get compile-time options for the
+    // usual combinations (gate and softplus on, with or without checkpoints)
+    if constexpr (sizeof(T) == 2 && N == 16 && (NT == 2 || NT == 4 || NT == 16)) {
+        const int fl = (fp.z ? 1 : 0) | (fp.softplus ? 2 : 0) | (fp.ckpt ? 4 : 0);
+        if (fl == 3) return launch_cfg<T, NT, N / NT, C::TT, C::NWC, C::STAGES, 3>(fp, stream);
+        if (fl == 7) return launch_cfg<T, NT, N / NT, C::TT, C::NWC, C::STAGES, 7>(fp, stream);
+    }
+    return launch_cfg<T, NT, N / NT, C::TT, C::NWC, C::STAGES, -1>(fp, stream);
 }
 
 template <typename T, int N, int NT>
