@@ -42,7 +42,7 @@ def _load():
         i = ctypes.c_int
         lib.ssm_oracle_fwd.argtypes = [i, i, i, i] + [dp] * 8 + [i, i, dp, dp, dp, i]
         lib.ssm_oracle_fwd.restype = i
-        lib.ssm_oracle_bwd.argtypes = [i, i, i, i] + [dp] * 8 + [i] + [dp] * 9 + [i]
+        lib.ssm_oracle_bwd.argtypes = [i, i, i, i] + [dp] * 8 + [i] + [dp] * 9 + [i, i]
         lib.ssm_oracle_bwd.restype = i
         lib.ssm_oracle_max_threads.restype = i
         _lib = lib
@@ -93,7 +93,7 @@ def step(state, u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softpl
     return out[..., 0], last
 
 
-def bwd(u, delta, A, B, C, D, z, delta_bias, delta_softplus, dout,
+def bwd(u, delta, A, B, C, D, z, delta_bias, delta_softplus, dout, zoh=False,
         nthreads: int = 0) -> Dict[str, np.ndarray]:
     """Returns a dict of float64 gradients: du, ddelta, dA, dB, dC and, where the
     matching input is given, dD, dz, ddelta_bias."""
@@ -110,7 +110,7 @@ def bwd(u, delta, A, B, C, D, z, delta_bias, delta_softplus, dout,
                                 _p(D), _p(z), _p(delta_bias), int(bool(delta_softplus)),
                                 _p(dout), _p(g["du"]), _p(g["ddelta"]), _p(g["dA"]),
                                 _p(g["dB"]), _p(g["dC"]), _p(g["dD"]), _p(g["dz"]),
-                                _p(g["ddelta_bias"]), int(nthreads))
+                                _p(g["ddelta_bias"]), int(bool(zoh)), int(nthreads))
     if rc != 0:
         raise MemoryError("oracle bwd: allocation failed")
     return {k: v for k, v in g.items() if v is not None}

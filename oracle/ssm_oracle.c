@@ -126,8 +126,20 @@ int ssm_oracle_fwd(int batch, int dim, int seqlen, int dstate,
     return 0;
 }
 
+/* d/dA of (exp(Δ a) - 1)/a, the zero-order-hold input factor: Δ² ψ(Δ a)
+ * with ψ(x) = (x e^x - (e^x - 1)) / x² = Σ_{j>=0} (j+1) x^j / (j+2)!,
+ * summed as a series near 0 where the closed form cancels. */
+static double zoh_dk_da(double dt, double a) {
+    double x = dt * a, psi;
+    if (fabs(x) < 1e-3)
+        psi = 0.5 + x * (1.0 / 3.0 + x * (1.0 / 8.0 + x * (1.0 / 30.0 + x / 144.0)));
+    else
+        psi = (x * exp(x) - expm1(x)) / (x * x);
+    return dt * dt * psi;
+}
+
 /*
- * Backward pass (the adjoint of ssm_oracle_fwd with zoh = 0 and h0 = 0),
+ * Backward pass (the adjoint of ssm_oracle_fwd with h0 = 0),
  * obtained by reverse-mode differentiation of the loop above.  The pages
  * give no backward formulas; only that the backward recomputes the states
  * ([SEL] §3.3), which this code does by re-running the forward recurrence
@@ -143,6 +155,9 @@ int ssm_oracle_fwd(int batch, int dim, int seqlen, int dstate,
  *   dA[d,n] += lam_t[n] Δ_t Ā_t[n] h_{t-1}[n]     dD[d] += gy_t u_t
  *   dB[b,n,t] += lam_t[n] Δ_t u_t                 dC[b,n,t] += gy_t h_t[n]
  *   dbias[d] += ddelta_t
+ * With zoh the input factor Δ_t above becomes k_t[n] = (Ā_t[n] - 1)/A[n]
+ * (Δ_t where A[n] = 0): du and dB use k, the B term of dΔ gains the factor
+ * dk/dΔ = Ā_t[n], and dA gains lam_t[n] B_t[n] u_t dk/dA (zoh_dk_da).
  * Gradients are written (not accumulated into).  dD / dz / dbias may be NULL
  * (and must be when the matching input is NULL).  Returns 0, or -1 if a
  * scratch allocation fails.
@@ -153,7 +168,7 @@ int ssm_oracle_bwd(int batch, int dim, int seqlen, int dstate,
                    const double *z, const double *delta_bias, int delta_softplus,
                    const double *dout, double *du, double *ddelta, double *dA,
                    double *dB, double *dC, double *dD, double *dz, double *dbias,
-                   int nthreads) {
+                   int zoh, int nthreads) {
     set_threads(nthreads);
     long npair = (long)batch * dim;
     size_t bcsz = (size_t)batch * dstate * seqlen;
@@ -213,9 +228,9 @@ int ssm_oracle_bwd(int batch, int dim, int seqlen, int dstate,
                 dts[t] = dt;
                 for (int n = 0; n < dstate; ++n) {
                     double abar = exp(dt * Ad[n]);
+                    double k = (zoh && Ad[n] != 0.0) ? expm1(dt * Ad[n]) / Ad[n] : dt;
                     hs[(size_t)(t + 1) * dstate + n] =
-                        abar * hs[(size_t)t * dstate + n] +
-                        dt * Bb[(size_t)n * seqlen + t] * ub[t];
+                        abar * hs[(size_t)t * dstate + n] + k * Bb[(size_t)n * seqlen + t] * ub[t];
                 }
             }
             /* reverse sweep */
@@ -242,13 +257,17 @@ int ssm_oracle_bwd(int batch, int dim, int seqlen, int dstate,
                     double Bt = Bb[(size_t)n * seqlen + t];
                     double Ct = Cb[(size_t)n * seqlen + t];
                     double abar = exp(dt * Ad[n]);
+                    int zn = zoh && Ad[n] != 0.0;
+                    double k = zn ? expm1(dt * Ad[n]) / Ad[n] : dt;   /* B̄ = k B */
+                    double dk_ddt = zoh ? abar : 1.0;
                     /* lam_t = C_t gy_t + Ā_{t+1} lam_{t+1}; lam[] holds
                        Ā_{t+1} lam_{t+1} on entry (see the update below) */
                     double l = Ct * gy + lam[n];
-                    dx += l * dt * Bt;
-                    ddt += l * (Ad[n] * abar * hprev[n] + Bt * x);
+                    dx += l * k * Bt;
+                    ddt += l * (Ad[n] * abar * hprev[n] + Bt * x * dk_ddt);
                     accA[n] += l * dt * abar * hprev[n];
-                    bB[(size_t)n * seqlen + t] += l * dt * x;
+                    if (zoh) accA[n] += l * Bt * x * zoh_dk_da(dt, Ad[n]);
+                    bB[(size_t)n * seqlen + t] += l * k * x;
                     bC[(size_t)n * seqlen + t] += gy * hcur[n];
                     lam[n] = abar * l; /* becomes Ā_t lam_t for step t-1 */
                 }

@@ -344,9 +344,9 @@ def test_threads_do_not_change_results():
 
 # ----------------------------------------------------------------- adjoint pins
 
-def _loss(c, dout, softplus):
+def _loss(c, dout, softplus, zoh=False):
     out, _ = oracle.fwd(c["u"], c["delta"], c["A"], c["B"], c["C"], c["D"], c["z"],
-                        c["delta_bias"], delta_softplus=softplus, nthreads=1)
+                        c["delta_bias"], delta_softplus=softplus, zoh=zoh, nthreads=1)
     return float((out * dout).sum())
 
 
@@ -381,6 +381,48 @@ def test_adjoint_matches_central_differences(softplus, gate, skip):
         scale = max(1.0, np.abs(fd).max())
         np.testing.assert_allclose(g[gname], fd, rtol=0, atol=1e-6 * scale,
                                    err_msg=f"gradient {gname}")
+
+
+@pytest.mark.parametrize("a_scale", [1.0, 1e-5, 0.0])
+def test_zoh_adjoint_matches_central_differences(a_scale):
+    """The zero-order-hold adjoint against central differences of the ZOH
+    forward (itself pinned to an RK4 solution), for ordinary A, for |Δ A|
+    small enough to take the series branch of dk/dA, and for A = 0 entries."""
+    c = rand_case(31, batch=1, dim=3, L=10, N=4)
+    c["A"] = c["A"] * a_scale
+    if a_scale == 0.0:
+        c["A"][0, 1] = -0.5            # mixed: zero and nonzero A in one channel
+    dout = rng(32).standard_normal(c["u"].shape)
+    g = oracle.bwd(c["u"], c["delta"], c["A"], c["B"], c["C"], c["D"], c["z"],
+                   c["delta_bias"], True, dout, zoh=True, nthreads=1)
+    for name, gname in GRAD_OF.items():
+        theta = c[name]
+        fd = np.zeros_like(theta)
+        for idx in np.ndindex(theta.shape):
+            old = theta[idx]
+            h = 1e-6 * max(1.0, abs(old))
+            theta[idx] = old + h
+            fp = _loss(c, dout, True, zoh=True)
+            theta[idx] = old - h
+            fm = _loss(c, dout, True, zoh=True)
+            theta[idx] = old
+            fd[idx] = (fp - fm) / (2 * h)
+        scale = max(1.0, np.abs(fd).max())
+        np.testing.assert_allclose(g[gname], fd, rtol=0, atol=1e-6 * scale,
+                                   err_msg=f"zoh gradient {gname}")
+
+
+def test_zoh_adjoint_differs_from_euler_b():
+    """A dropped ZOH term would leave the gradients equal to the B̄ = ΔB ones;
+    at |ΔA| ~ 1 they must differ."""
+    c = rand_case(33, batch=1, dim=2, L=6, N=4)
+    dout = rng(34).standard_normal(c["u"].shape)
+    g0 = oracle.bwd(c["u"], c["delta"], c["A"], c["B"], c["C"], c["D"], c["z"],
+                    c["delta_bias"], True, dout, zoh=False)
+    g1 = oracle.bwd(c["u"], c["delta"], c["A"], c["B"], c["C"], c["D"], c["z"],
+                    c["delta_bias"], True, dout, zoh=True)
+    for k in ("du", "ddelta", "dA", "dB"):
+        assert np.abs(g0[k] - g1[k]).max() > 1e-3 * np.abs(g0[k]).max(), k
 
 
 def test_adjoint_directional_derivative_larger_case():
