@@ -77,6 +77,20 @@ typedef struct {
     ssm_dtype_t io_dtype; /* dtype of u, delta, z, B, C, out, dout */
 } ssm_shape_t;
 
+/* Discretisation of the input matrix (booiljung.github.io, "3.2 선택적
+ * 스캔(Selective Scan) 알고리즘", §2.1 prints the zero-order hold
+ * B̄ = (ΔA)^-1 (exp(ΔA) - I) ΔB; with diagonal A it is elementwise). */
+typedef enum {
+    SSM_DISC_DELTA_B = 0, /* B̄ = Δ B: what every entry point without _ex uses */
+    SSM_DISC_ZOH = 1      /* B̄ = (exp(Δ A) - 1) / A · B, Δ B where A = 0 (its limit) */
+} ssm_discretization_t;
+
+/* Options of the _ex entry points. */
+typedef struct {
+    int delta_softplus;                  /* nonzero: Δ = softplus(delta + delta_bias) */
+    ssm_discretization_t discretization;
+} ssm_options_t;
+
 /* Steps between two saved states in the forward's checkpoint buffer.  The
  * backward recomputes each such window of steps once from its saved state. */
 #define SSM_CKPT_CHUNK 8
@@ -114,6 +128,22 @@ ssm_status_t ssm_selective_scan_fwd(const ssm_shape_t *shape,
                                     const float *delta_bias, int delta_softplus,
                                     void *out, float *last_state, float *ckpt,
                                     void *stream);
+
+/*
+ * ssm_selective_scan_fwd with options: opts->delta_softplus replaces
+ * delta_softplus and opts->discretization selects B̄ (SSM_DISC_ZOH is served
+ * by the general kernel).  Checkpoints written with SSM_DISC_ZOH must be
+ * passed to a backward with SSM_DISC_ZOH.
+ * Errors: as ssm_selective_scan_fwd, plus SSM_ERR_INVALID_ARG for a NULL
+ * opts or an unknown discretization.
+ */
+ssm_status_t ssm_selective_scan_fwd_ex(const ssm_shape_t *shape, const ssm_options_t *opts,
+                                       const void *u, const void *delta,
+                                       const float *A, const void *B, const void *C,
+                                       const float *D, const void *z,
+                                       const float *delta_bias,
+                                       void *out, float *last_state, float *ckpt,
+                                       void *stream);
 
 /*
  * Bytes of device scratch that ssm_selective_scan_bwd needs: 0 when the
@@ -218,6 +248,30 @@ ssm_status_t ssm_selective_state_update(const ssm_shape_t *shape, float *state,
                                         const float *D, const void *z,
                                         const float *delta_bias, int delta_softplus,
                                         void *out, void *stream);
+
+/*
+ * ssm_selective_scan_bwd with options (see ssm_selective_scan_fwd_ex): the
+ * adjoint of the forward with the same options.  With SSM_DISC_ZOH, du and
+ * dB use the ZOH factor (Ā - 1)/A in place of Δ, the B term of dΔ carries
+ * dB̄/dΔ = Ā B, and dA gains the derivative of (Ā - 1)/A with respect to A.
+ */
+ssm_status_t ssm_selective_scan_bwd_ex(const ssm_shape_t *shape, const ssm_options_t *opts,
+                                       const void *u, const void *delta,
+                                       const float *A, const void *B, const void *C,
+                                       const float *D, const void *z,
+                                       const float *delta_bias, const void *dout,
+                                       const float *ckpt,
+                                       float *du, float *ddelta, float *dA,
+                                       float *dB, float *dC, float *dD, float *dz,
+                                       float *ddelta_bias,
+                                       void *scratch, size_t scratch_bytes, void *stream);
+
+/* ssm_selective_state_update with options (see ssm_selective_scan_fwd_ex). */
+ssm_status_t ssm_selective_state_update_ex(const ssm_shape_t *shape, const ssm_options_t *opts,
+                                           float *state, const void *u, const void *delta,
+                                           const float *A, const void *B, const void *C,
+                                           const float *D, const void *z,
+                                           const float *delta_bias, void *out, void *stream);
 
 /*
  * Synchronises `stream`, then reports (and clears) the device-side error word

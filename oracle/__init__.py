@@ -82,14 +82,15 @@ def fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True,
     return out, last
 
 
-def step(state, u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True):
+def step(state, u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=True,
+         zoh=False):
     """One step of the recurrence from `state` ([b,d,N]): u, delta, z are
     [b,d], B, C [b,N].  It is the forward over a single time step started
     from h0 = state.  Returns (out [b,d], new_state [b,d,N]) in float64."""
     u, delta, B, C = (np.asarray(x, dtype=np.float64) for x in (u, delta, B, C))
     out, last = fwd(u[..., None], delta[..., None], A, B[..., None], C[..., None], D,
                     None if z is None else np.asarray(z, dtype=np.float64)[..., None],
-                    delta_bias, delta_softplus, h0=state)
+                    delta_bias, delta_softplus, zoh=zoh, h0=state)
     return out[..., 0], last
 
 

@@ -121,6 +121,14 @@ int n_ckpt(const ssm_shape_t *s) { return (s->seqlen + SSM_CKPT_CHUNK - 1) / SSM
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15) == 0; }
 
+ssm_status_t check_options(const ssm_options_t *o) {
+    if (!o) return fail(SSM_ERR_INVALID_ARG, "options is NULL");
+    if (o->discretization != SSM_DISC_DELTA_B && o->discretization != SSM_DISC_ZOH)
+        return fail(SSM_ERR_INVALID_ARG, "discretization %d is not SSM_DISC_DELTA_B or SSM_DISC_ZOH",
+                    (int)o->discretization);
+    return SSM_OK;
+}
+
 }  // namespace
 
 ssm_status_t ssm::set_last_error(ssm_status_t status, const char *msg) {
@@ -150,11 +158,13 @@ ssm_status_t ssm_selective_scan_bwd_scratch_bytes(const ssm_shape_t *shape, int 
     return ok();
 }
 
-ssm_status_t ssm_selective_scan_fwd(const ssm_shape_t *shape, const void *u, const void *delta,
-                                    const float *A, const void *B, const void *C, const float *D,
-                                    const void *z, const float *delta_bias, int delta_softplus,
-                                    void *out, float *last_state, float *ckpt, void *stream) {
+ssm_status_t ssm_selective_scan_fwd_ex(const ssm_shape_t *shape, const ssm_options_t *opts,
+                                       const void *u, const void *delta, const float *A,
+                                       const void *B, const void *C, const float *D, const void *z,
+                                       const float *delta_bias, void *out, float *last_state,
+                                       float *ckpt, void *stream) {
     SSM_TRY(check_shape(shape));
+    SSM_TRY(check_options(opts));
     const size_t es = esize(shape->io_dtype);
     SSM_TRY(check_ptr(u, "u", es, true));
     SSM_TRY(check_ptr(delta, "delta", es, true));
@@ -175,7 +185,8 @@ ssm_status_t ssm_selective_scan_fwd(const ssm_shape_t *shape, const void *u, con
     p.delta_bias = delta_bias; p.out = out; p.last_state = last_state; p.ckpt = ckpt;
     p.batch = shape->batch; p.dim = shape->dim; p.L = shape->seqlen; p.N = shape->dstate;
     p.n_ckpt = n_ckpt(shape);
-    p.softplus = delta_softplus != 0;
+    p.softplus = opts->delta_softplus != 0;
+    p.zoh = opts->discretization == SSM_DISC_ZOH;
     p.io_bf16 = shape->io_dtype == SSM_BF16;
     p.vec_ok = ((size_t)shape->seqlen * es) % 16 == 0 && aligned16(u) && aligned16(delta) &&
                aligned16(B) && aligned16(C) && aligned16(out) && (!z || aligned16(z));
@@ -184,14 +195,15 @@ ssm_status_t ssm_selective_scan_fwd(const ssm_shape_t *shape, const void *u, con
     return ok();
 }
 
-ssm_status_t ssm_selective_scan_bwd(const ssm_shape_t *shape, const void *u, const void *delta,
-                                    const float *A, const void *B, const void *C, const float *D,
-                                    const void *z, const float *delta_bias, int delta_softplus,
-                                    const void *dout, const float *ckpt, float *du, float *ddelta,
-                                    float *dA, float *dB, float *dC, float *dD, float *dz,
-                                    float *ddelta_bias, void *scratch, size_t scratch_bytes,
-                                    void *stream) {
+ssm_status_t ssm_selective_scan_bwd_ex(const ssm_shape_t *shape, const ssm_options_t *opts,
+                                       const void *u, const void *delta, const float *A,
+                                       const void *B, const void *C, const float *D, const void *z,
+                                       const float *delta_bias, const void *dout, const float *ckpt,
+                                       float *du, float *ddelta, float *dA, float *dB, float *dC,
+                                       float *dD, float *dz, float *ddelta_bias, void *scratch,
+                                       size_t scratch_bytes, void *stream) {
     SSM_TRY(check_shape(shape));
+    SSM_TRY(check_options(opts));
     const size_t es = esize(shape->io_dtype);
     SSM_TRY(check_ptr(u, "u", es, true));
     SSM_TRY(check_ptr(delta, "delta", es, true));
@@ -234,7 +246,8 @@ ssm_status_t ssm_selective_scan_bwd(const ssm_shape_t *shape, const void *u, con
         fp.u = u; fp.delta = delta; fp.A = A; fp.B = B; fp.C = C; fp.D = D; fp.z = z;
         fp.delta_bias = delta_bias; fp.out = nullptr; fp.last_state = nullptr; fp.ckpt = ck;
         fp.batch = shape->batch; fp.dim = shape->dim; fp.L = shape->seqlen; fp.N = shape->dstate;
-        fp.n_ckpt = nck; fp.softplus = delta_softplus != 0;
+        fp.n_ckpt = nck; fp.softplus = opts->delta_softplus != 0;
+        fp.zoh = opts->discretization == SSM_DISC_ZOH;
         fp.io_bf16 = shape->io_dtype == SSM_BF16; fp.vec_ok = vec_ok;
         cudaError_t e = ssm::launch_fwd(fp, true, st);
         if (e != cudaSuccess) return cuda_fail(e, "ssm_selective_scan_bwd state pass");
@@ -255,19 +268,21 @@ ssm_status_t ssm_selective_scan_bwd(const ssm_shape_t *shape, const void *u, con
     p.du = du; p.ddelta = ddelta; p.dA = dA; p.dB = dB; p.dC = dC; p.dD = dD; p.dz = dz;
     p.ddelta_bias = ddelta_bias;
     p.batch = shape->batch; p.dim = shape->dim; p.L = shape->seqlen; p.N = shape->dstate;
-    p.n_ckpt = nck; p.softplus = delta_softplus != 0;
+    p.n_ckpt = nck; p.softplus = opts->delta_softplus != 0;
+    p.zoh = opts->discretization == SSM_DISC_ZOH;
     p.io_bf16 = shape->io_dtype == SSM_BF16; p.vec_ok = vec_ok;
     e = ssm::launch_bwd(p, st);
     if (e != cudaSuccess) return cuda_fail(e, "ssm_selective_scan_bwd launch");
     return ok();
 }
 
-ssm_status_t ssm_selective_state_update(const ssm_shape_t *shape, float *state, const void *u,
-                                        const void *delta, const float *A, const void *B,
-                                        const void *C, const float *D, const void *z,
-                                        const float *delta_bias, int delta_softplus, void *out,
-                                        void *stream) {
+ssm_status_t ssm_selective_state_update_ex(const ssm_shape_t *shape, const ssm_options_t *opts,
+                                           float *state, const void *u, const void *delta,
+                                           const float *A, const void *B, const void *C,
+                                           const float *D, const void *z, const float *delta_bias,
+                                           void *out, void *stream) {
     SSM_TRY(check_shape(shape));
+    SSM_TRY(check_options(opts));
     if (shape->seqlen != 1)
         return fail(SSM_ERR_INVALID_ARG, "a single step needs seqlen == 1 (got %d)", shape->seqlen);
     if (shape->batch > 65535)
@@ -290,12 +305,45 @@ ssm_status_t ssm_selective_state_update(const ssm_shape_t *shape, float *state, 
     p.state = state; p.u = u; p.delta = delta; p.A = A; p.B = B; p.C = C; p.D = D; p.z = z;
     p.delta_bias = delta_bias; p.out = out;
     p.P = (long long)shape->batch * shape->dim; p.dim = shape->dim; p.N = shape->dstate;
-    p.softplus = delta_softplus != 0;
+    p.softplus = opts->delta_softplus != 0;
+    p.zoh = opts->discretization == SSM_DISC_ZOH;
     p.io_bf16 = shape->io_dtype == SSM_BF16;
     p.vec_ok = aligned16(state) && aligned16(A) && aligned16(B) && aligned16(C);
     cudaError_t e = ssm::launch_state_update(p, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "ssm_selective_state_update launch");
     return ok();
+}
+
+ssm_status_t ssm_selective_scan_fwd(const ssm_shape_t *shape, const void *u, const void *delta,
+                                    const float *A, const void *B, const void *C, const float *D,
+                                    const void *z, const float *delta_bias, int delta_softplus,
+                                    void *out, float *last_state, float *ckpt, void *stream) {
+    const ssm_options_t o = {delta_softplus, SSM_DISC_DELTA_B};
+    return ssm_selective_scan_fwd_ex(shape, &o, u, delta, A, B, C, D, z, delta_bias, out,
+                                     last_state, ckpt, stream);
+}
+
+ssm_status_t ssm_selective_scan_bwd(const ssm_shape_t *shape, const void *u, const void *delta,
+                                    const float *A, const void *B, const void *C, const float *D,
+                                    const void *z, const float *delta_bias, int delta_softplus,
+                                    const void *dout, const float *ckpt, float *du, float *ddelta,
+                                    float *dA, float *dB, float *dC, float *dD, float *dz,
+                                    float *ddelta_bias, void *scratch, size_t scratch_bytes,
+                                    void *stream) {
+    const ssm_options_t o = {delta_softplus, SSM_DISC_DELTA_B};
+    return ssm_selective_scan_bwd_ex(shape, &o, u, delta, A, B, C, D, z, delta_bias, dout, ckpt,
+                                     du, ddelta, dA, dB, dC, dD, dz, ddelta_bias, scratch,
+                                     scratch_bytes, stream);
+}
+
+ssm_status_t ssm_selective_state_update(const ssm_shape_t *shape, float *state, const void *u,
+                                        const void *delta, const float *A, const void *B,
+                                        const void *C, const float *D, const void *z,
+                                        const float *delta_bias, int delta_softplus, void *out,
+                                        void *stream) {
+    const ssm_options_t o = {delta_softplus, SSM_DISC_DELTA_B};
+    return ssm_selective_state_update_ex(shape, &o, state, u, delta, A, B, C, D, z, delta_bias,
+                                         out, stream);
 }
 
 ssm_status_t ssm_device_error_status(void *stream) {

@@ -54,7 +54,10 @@ struct BwdSmem {
     static constexpr size_t bytes = sizeof(float) * kTotal;
 };
 
-template <typename T, int NT, int NS, int G, int W>
+// ZOH: the adjoint of the zero-order-hold forward (B̄ = φ(ΔA) Δ B): du and
+// dB use φ Δ, the B term of dΔ carries dk/dΔ = Ā, and dA gains
+// λ B u Δ² ψ(ΔA) (zoh_phi, zoh_psi).
+template <typename T, int NT, int NS, int G, int W, bool ZOH>
 __global__ void __launch_bounds__(NT * G)
 bwd_kernel(const BwdParams p) {
     using S = BwdSmem<NT, NS, G, W>;
@@ -165,7 +168,8 @@ bwd_kernel(const BwdParams p) {
 #pragma unroll
                 for (int s = 0; s < NS; ++s) {
                     const float a = ex2(dt * A2[s]);
-                    h[s] = fmaf(a, h[s], du * sB[t * NSB + g * NS + s]);
+                    const float k = ZOH ? zoh_phi(dt * Aw[s], a) * du : du;
+                    h[s] = fmaf(a, h[s], k * sB[t * NSB + g * NS + s]);
                     acc = fmaf(sC[t * NSB + g * NS + s], h[s], acc);
                 }
                 sP0[(g * G + c) * W + t] = acc;
@@ -217,7 +221,8 @@ bwd_kernel(const BwdParams p) {
                     for (int s = 0; s < NS; ++s) {
                         ab[t][s] = ex2(dt * A2[s]);
                         hp[t][s] = hw[s];
-                        hw[s] = fmaf(ab[t][s], hw[s], du * sB[t * NSB + g * NS + s]);
+                        const float k = ZOH ? zoh_phi(dt * Aw[s], ab[t][s]) * du : du;
+                        hw[s] = fmaf(ab[t][s], hw[s], k * sB[t * NSB + g * NS + s]);
                     }
                 }
             }
@@ -225,6 +230,9 @@ bwd_kernel(const BwdParams p) {
             for (int t = W - 1; t >= 0; --t) {
                 const float gy = sGy[c * CS + w * W + t];
                 const float dt = sDt[c * WS + t], du = sDu[c * WS + t];
+                const float xu = ZOH ? sU[c * WS + t] : 0.f;
+                // sa: Σ over the lane's states of the dΔ terms (through Ā, and
+                // with ZOH through B̄ too); sb: Σ λ B (ZOH: Σ λ φ B), the du term / Δ
                 float sa = 0.f, sb = 0.f;
                 float dBv[NS], dCv[NS];
 #pragma unroll
@@ -232,12 +240,20 @@ bwd_kernel(const BwdParams p) {
                     const float Bt = sB[t * NSB + g * NS + s], Ct = sC[t * NSB + g * NS + s];
                     const float l = fmaf(anext[s], lam[s], Ct * gy);
                     const float a = ab[t][s], hv = hp[t][s];
-                    const float hcur = fmaf(a, hv, du * Bt);
+                    const float phi = ZOH ? zoh_phi(dt * Aw[s], a) : 1.f;
+                    const float hcur = fmaf(a, hv, phi * du * Bt);
                     const float wv = l * a * hv;
                     dA_acc[s] = fmaf(dt, wv, dA_acc[s]);
                     sa = fmaf(Aw[s], wv, sa);
-                    sb = fmaf(l, Bt, sb);
-                    dBv[s] = l * du;
+                    if (ZOH) {
+                        const float lB = l * Bt;
+                        dA_acc[s] = fmaf(lB * xu, dt * dt * zoh_psi(dt * Aw[s], a), dA_acc[s]);
+                        sa = fmaf(xu * a, lB, sa);
+                        sb = fmaf(lB, phi, sb);
+                    } else {
+                        sb = fmaf(l, Bt, sb);
+                    }
+                    dBv[s] = l * phi * du;
                     dCv[s] = gy * hcur;
                     lam[s] = l;
                     anext[s] = a;
@@ -265,7 +281,7 @@ bwd_kernel(const BwdParams p) {
                     }
                     const float dt = sDt[c * WS + t], x = sU[c * WS + t];
                     const float gy = sGy[c * CS + w * W + t];
-                    const float dDelta = fmaf(x, sb, sa);
+                    const float dDelta = ZOH ? sa : fmaf(x, sb, sa);
                     const float ddr = p.softplus ? dDelta * sigmoid(sR[c * WS + t]) : dDelta;
                     const size_t off = (row_bd0 + d) * (size_t)L + tg;
                     p.du[off] = fmaf(gy, Dd, dt * sb);
@@ -308,10 +324,10 @@ bwd_kernel(const BwdParams p) {
     }
 }
 
-template <typename T, int NT, int NS, int G, int W>
+template <typename T, int NT, int NS, int G, int W, bool ZOH>
 static cudaError_t launch_bwd_cfg(const BwdParams &p, cudaStream_t stream) {
     using S = BwdSmem<NT, NS, G, W>;
-    auto kern = bwd_kernel<T, NT, NS, G, W>;
+    auto kern = bwd_kernel<T, NT, NS, G, W, ZOH>;
     static bool attr_done = false;
     if (!attr_done) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -324,17 +340,22 @@ static cudaError_t launch_bwd_cfg(const BwdParams &p, cudaStream_t stream) {
     return cudaGetLastError();
 }
 
-template <typename T>
-static cudaError_t launch_bwd_t(const BwdParams &p, cudaStream_t stream) {
+template <typename T, bool ZOH>
+static cudaError_t launch_bwd_tz(const BwdParams &p, cudaStream_t stream) {
     switch (p.N) {
-    case 1: return launch_bwd_cfg<T, 1, 1, 64, 8>(p, stream);
-    case 2: return launch_bwd_cfg<T, 1, 2, 64, 8>(p, stream);
-    case 4: return launch_bwd_cfg<T, 1, 4, 64, 8>(p, stream);
-    case 8: return launch_bwd_cfg<T, 2, 4, 32, 8>(p, stream);
-    case 16: return launch_bwd_cfg<T, 4, 4, 32, 8>(p, stream);
-    case 32: return launch_bwd_cfg<T, 8, 4, 16, 8>(p, stream);
+    case 1: return launch_bwd_cfg<T, 1, 1, 64, 8, ZOH>(p, stream);
+    case 2: return launch_bwd_cfg<T, 1, 2, 64, 8, ZOH>(p, stream);
+    case 4: return launch_bwd_cfg<T, 1, 4, 64, 8, ZOH>(p, stream);
+    case 8: return launch_bwd_cfg<T, 2, 4, 32, 8, ZOH>(p, stream);
+    case 16: return launch_bwd_cfg<T, 4, 4, 32, 8, ZOH>(p, stream);
+    case 32: return launch_bwd_cfg<T, 8, 4, 16, 8, ZOH>(p, stream);
     default: return cudaErrorInvalidValue;
     }
+}
+
+template <typename T>
+static cudaError_t launch_bwd_t(const BwdParams &p, cudaStream_t stream) {
+    return p.zoh ? launch_bwd_tz<T, true>(p, stream) : launch_bwd_tz<T, false>(p, stream);
 }
 
 cudaError_t launch_bwd(const BwdParams &p, cudaStream_t stream) {

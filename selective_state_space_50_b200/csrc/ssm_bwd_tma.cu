@@ -682,7 +682,7 @@ constexpr int kBwdWarpsBf16 = SSM_BWD_WARPS_BF16, kBwdWarpsF32 = SSM_BWD_WARPS_F
 bool try_launch_bwd_tma(const BwdParams &bp, cudaStream_t stream, cudaError_t *err) {
     static const char *force = getenv("SSM_BWD_KERNEL");
     if (force && !strcmp(force, "general")) return false;
-    if (!bp.vec_ok || bp.N != 16 || !bp.ckpt) return false;
+    if (!bp.vec_ok || bp.N != 16 || !bp.ckpt || bp.zoh) return false;   // zero-order hold: general kernel
     if (!aligned_to(bp.ckpt, 16) || !aligned_to(bp.dB, 16) || !aligned_to(bp.dC, 16) ||
         !aligned_to(bp.du, 8) || !aligned_to(bp.ddelta, 8) || (bp.dz && !aligned_to(bp.dz, 8)))
         return false;

@@ -102,6 +102,28 @@ __device__ __forceinline__ float2 ex2_poly2(float2 x) {
                        __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
 
+// ---- zero-order-hold discretisation ----------------------------------------
+// With diagonal A the ZOH input matrix is B̄ = (Ā - 1)/A · B = φ(x) Δ B with
+// x = Δ A and φ(x) = (e^x - 1)/x (→ 1 as A → 0, the B̄ = ΔB limit).  Given
+// a = e^x, φ is (a - 1)/x except near 0, where that difference cancels and
+// the Taylor series 1 + x/2 + x²/6 + ... + x⁵/720 is used (truncation below
+// 3e-10 for |x| < 0.1).
+__device__ __forceinline__ float zoh_phi(float x, float a) {
+    if (fabsf(x) < 0.1f)
+        return fmaf(x, fmaf(x, fmaf(x, fmaf(x, fmaf(x, 1.f / 720.f, 1.f / 120.f), 1.f / 24.f), 1.f / 6.f),
+                            0.5f), 1.f);
+    return __fdividef(a - 1.f, x);
+}
+
+// ψ(x) = (x e^x - (e^x - 1)) / x², so that d/dA of the ZOH factor
+// (e^{ΔA} - 1)/A is Δ² ψ(ΔA); its series near 0 is
+// 1/2 + x/3 + x²/8 + x³/30 + x⁴/144 (truncation below 2e-8 for |x| < 0.1).
+__device__ __forceinline__ float zoh_psi(float x, float a) {
+    if (fabsf(x) < 0.1f)
+        return fmaf(x, fmaf(x, fmaf(x, fmaf(x, 1.f / 144.f, 1.f / 30.f), 1.f / 8.f), 1.f / 3.f), 0.5f);
+    return __fdividef(fmaf(x, a, 1.f - a), x * x);
+}
+
 // ---- io element types -------------------------------------------------------
 
 template <typename T> struct IO;

@@ -64,8 +64,9 @@ struct FwdSmem {
 };
 
 // MODE 0: full forward.  MODE 1: states only (writes ckpt / last_state, no
-// readout), used by the backward when no checkpoints were given.
-template <typename T, int NT, int NS, int G, int TT, int MODE>
+// readout), used by the backward when no checkpoints were given.  ZOH: the
+// zero-order-hold input matrix B̄ = φ(ΔA) Δ B (zoh_phi) instead of Δ B.
+template <typename T, int NT, int NS, int G, int TT, int MODE, bool ZOH>
 __global__ void __launch_bounds__(NT * G)
 fwd_kernel(const FwdParams p) {
     using S = FwdSmem<T, NT, NS, G, TT>;
@@ -191,8 +192,10 @@ fwd_kernel(const FwdParams p) {
                 float acc = 0.f;
 #pragma unroll
                 for (int s = 0; s < NS; ++s) {
-                    const float a = ex2(dts[i] * A2[s]);
-                    h[s] = fmaf(a, h[s], dus[i] * bv[s]);
+                    const float arg = dts[i] * A2[s];
+                    const float a = ex2(arg);
+                    const float k = ZOH ? zoh_phi(arg * 0.69314718f, a) * dus[i] : dus[i];
+                    h[s] = fmaf(a, h[s], k * bv[s]);
                     if (MODE == 0) acc = fmaf(cv[s], h[s], acc);
                 }
                 yv[i] = acc;
@@ -257,10 +260,10 @@ fwd_kernel(const FwdParams p) {
 
 // ---------------------------------------------------------------- launch
 
-template <typename T, int NT, int NS, int G, int TT, int MODE>
+template <typename T, int NT, int NS, int G, int TT, int MODE, bool ZOH>
 static cudaError_t launch_fwd_cfg(const FwdParams &p, cudaStream_t stream) {
     using S = FwdSmem<T, NT, NS, G, TT>;
-    auto kern = fwd_kernel<T, NT, NS, G, TT, MODE>;
+    auto kern = fwd_kernel<T, NT, NS, G, TT, MODE, ZOH>;
     static bool attr_done = false;  // per instance; benign race (idempotent)
     if (!attr_done) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -275,24 +278,29 @@ static cudaError_t launch_fwd_cfg(const FwdParams &p, cudaStream_t stream) {
 
 // Picks the lane split for dstate N.  With few (b, d) pairs (long sequences,
 // small batch) every state gets its own lane to keep enough warps resident.
-template <typename T, int MODE>
-static cudaError_t launch_fwd_t(const FwdParams &p, cudaStream_t stream) {
+template <typename T, int MODE, bool ZOH>
+static cudaError_t launch_fwd_tz(const FwdParams &p, cudaStream_t stream) {
     const long pairs = (long)p.batch * p.dim;
     const bool few = pairs < 4096;
     constexpr int TT = 32;
     switch (p.N) {
-    case 1: return launch_fwd_cfg<T, 1, 1, 128, TT, MODE>(p, stream);
-    case 2: return launch_fwd_cfg<T, 1, 2, 128, TT, MODE>(p, stream);
-    case 4: return few ? launch_fwd_cfg<T, 4, 1, 32, TT, MODE>(p, stream)
-                       : launch_fwd_cfg<T, 1, 4, 128, TT, MODE>(p, stream);
-    case 8: return few ? launch_fwd_cfg<T, 8, 1, 16, TT, MODE>(p, stream)
-                       : launch_fwd_cfg<T, 2, 4, 64, TT, MODE>(p, stream);
-    case 16: return few ? launch_fwd_cfg<T, 16, 1, 8, TT, MODE>(p, stream)
-                        : launch_fwd_cfg<T, 4, 4, 32, TT, MODE>(p, stream);
-    case 32: return few ? launch_fwd_cfg<T, 16, 2, 8, TT, MODE>(p, stream)
-                        : launch_fwd_cfg<T, 8, 4, 16, TT, MODE>(p, stream);
+    case 1: return launch_fwd_cfg<T, 1, 1, 128, TT, MODE, ZOH>(p, stream);
+    case 2: return launch_fwd_cfg<T, 1, 2, 128, TT, MODE, ZOH>(p, stream);
+    case 4: return few ? launch_fwd_cfg<T, 4, 1, 32, TT, MODE, ZOH>(p, stream)
+                       : launch_fwd_cfg<T, 1, 4, 128, TT, MODE, ZOH>(p, stream);
+    case 8: return few ? launch_fwd_cfg<T, 8, 1, 16, TT, MODE, ZOH>(p, stream)
+                       : launch_fwd_cfg<T, 2, 4, 64, TT, MODE, ZOH>(p, stream);
+    case 16: return few ? launch_fwd_cfg<T, 16, 1, 8, TT, MODE, ZOH>(p, stream)
+                        : launch_fwd_cfg<T, 4, 4, 32, TT, MODE, ZOH>(p, stream);
+    case 32: return few ? launch_fwd_cfg<T, 16, 2, 8, TT, MODE, ZOH>(p, stream)
+                        : launch_fwd_cfg<T, 8, 4, 16, TT, MODE, ZOH>(p, stream);
     default: return cudaErrorInvalidValue;
     }
+}
+
+template <typename T, int MODE>
+static cudaError_t launch_fwd_t(const FwdParams &p, cudaStream_t stream) {
+    return p.zoh ? launch_fwd_tz<T, MODE, true>(p, stream) : launch_fwd_tz<T, MODE, false>(p, stream);
 }
 
 cudaError_t launch_fwd(const FwdParams &p, bool states_only, cudaStream_t stream) {

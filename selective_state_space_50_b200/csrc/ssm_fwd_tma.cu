@@ -590,7 +590,7 @@ bool nt_valid(int N, int nt) {
 // Returns true (and launches) when the TMA path applies; false means the
 // caller should use the general kernel.
 bool try_launch_fwd_tma(const FwdParams &fp, cudaStream_t stream, cudaError_t *err) {
-    if (!fp.vec_ok || !fp.out) return false;
+    if (!fp.vec_ok || !fp.out || fp.zoh) return false;   // zero-order hold: general kernel
     if (fp.N != 8 && fp.N != 16 && fp.N != 32) return false;
     if (!tma_available()) return false;
     const long long P = (long long)fp.batch * fp.dim;

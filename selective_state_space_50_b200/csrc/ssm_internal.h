@@ -20,6 +20,7 @@ struct FwdParams {
     float *last_state, *ckpt;
     int batch, dim, L, N, n_ckpt;
     int softplus;
+    int zoh;      // zero-order-hold B̄ (general kernels only)
     bool io_bf16;
     bool vec_ok;  // every [.., L] row starts 16-byte aligned
 };
@@ -36,6 +37,7 @@ struct BwdParams {
     float *du, *ddelta, *dA, *dB, *dC, *dD, *dz, *ddelta_bias;
     int batch, dim, L, N, n_ckpt;
     int softplus;
+    int zoh;      // zero-order-hold B̄ (general kernel only)
     bool io_bf16;
     bool vec_ok;
 };
@@ -52,6 +54,7 @@ struct StepParams {
     long long P;                   // batch * dim
     int dim, N;
     int softplus;
+    int zoh;                       // zero-order-hold B̄
     bool io_bf16;
     bool vec_ok;                   // state, A, B, C 16-byte aligned (vector access)
 };

@@ -1,6 +1,7 @@
 // Single-step recurrent update (decoding one token): for each (batch b,
 // channel d) the state advances by one time step in place,
-//   Δ = softplus(delta + bias[d]),  h[n] ← exp(Δ A[d,n]) h[n] + Δ B[n] u,
+//   Δ = softplus(delta + bias[d]),  h[n] ← exp(Δ A[d,n]) h[n] + Δ B[n] u
+//   (zero-order hold: (exp(Δ A[d,n]) - 1)/A[d,n] B[n] u in the last term),
 //   y = Σ_n C[n] h[n] + D[d] u,     out = y · z σ(z),
 // the recurrent form of the selective SSM (정보관리기술사 학습 노트, "상태공간
 // 모델(SSM)과 Mamba 아키텍처" §2: h_t = Ā h_{t-1} + B̄ x_t, y_t = C h_t;
@@ -106,7 +107,8 @@ __global__ void __launch_bounds__(256) state_update_kernel(const StepParams p) {
 #pragma unroll
         for (int i = 0; i < SPT; ++i) {
             const float a = ex2(dt * (a2[k][i] * SSM_LOG2E));
-            h[k][i] = fmaf(a, h[k][i], du * bb[i]);
+            const float coef = p.zoh ? zoh_phi(dt * a2[k][i], a) * du : du;   // B̄ u / B
+            h[k][i] = fmaf(a, h[k][i], coef * bb[i]);
             y = fmaf(cc[i], h[k][i], y);
         }
 #pragma unroll

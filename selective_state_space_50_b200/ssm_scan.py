@@ -25,7 +25,10 @@ CKPT_CHUNK = 8  # SSM_CKPT_CHUNK in include/ssm_scan.h
 EXPORTS = ("ssm_version", "ssm_last_error_string", "ssm_selective_scan_ckpt_bytes",
            "ssm_selective_scan_fwd", "ssm_selective_scan_bwd_scratch_bytes",
            "ssm_selective_scan_bwd", "ssm_device_error_status",
-           "ssm_selective_scan_bwd_noalloc", "ssm_selective_state_update")
+           "ssm_selective_scan_bwd_noalloc", "ssm_selective_state_update",
+           "ssm_selective_scan_fwd_ex", "ssm_selective_scan_bwd_ex",
+           "ssm_selective_state_update_ex")
+SSM_DISC_DELTA_B, SSM_DISC_ZOH = 0, 1
 NOALLOC_SCRATCH_BYTES = 32 << 20  # SSM_NOALLOC_SCRATCH_BYTES in include/ssm_scan.h
 
 
@@ -38,6 +41,14 @@ class SSMError(RuntimeError):
 class Shape(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int), ("dim", ctypes.c_int), ("seqlen", ctypes.c_int),
                 ("dstate", ctypes.c_int), ("io_dtype", ctypes.c_int)]
+
+
+class Options(ctypes.Structure):
+    _fields_ = [("delta_softplus", ctypes.c_int), ("discretization", ctypes.c_int)]
+
+
+def _opts(delta_softplus: bool, zoh: bool) -> Options:
+    return Options(int(bool(delta_softplus)), SSM_DISC_ZOH if zoh else SSM_DISC_DELTA_B)
 
 
 _lib = None
@@ -70,6 +81,13 @@ def load_library(path: str = LIB_PATH):
     lib.ssm_selective_scan_bwd_noalloc.restype = i
     lib.ssm_selective_state_update.argtypes = [sp] + [vp] * 9 + [i] + [vp] * 2
     lib.ssm_selective_state_update.restype = i
+    op = ctypes.POINTER(Options)
+    lib.ssm_selective_scan_fwd_ex.argtypes = [sp, op] + [vp] * 12
+    lib.ssm_selective_scan_fwd_ex.restype = i
+    lib.ssm_selective_scan_bwd_ex.argtypes = [sp, op] + [vp] * 19 + [sz, vp]
+    lib.ssm_selective_scan_bwd_ex.restype = i
+    lib.ssm_selective_state_update_ex.argtypes = [sp, op] + [vp] * 11
+    lib.ssm_selective_state_update_ex.restype = i
     _lib = lib
     return lib
 
@@ -124,8 +142,16 @@ def _shape_of(u: torch.Tensor, A: torch.Tensor) -> Shape:
 
 
 def fwd_raw(shape: Shape, u, delta, A, B, C, D, z, delta_bias, delta_softplus: bool,
-            out, last_state, ckpt, stream=None):
-    """Direct C-ABI call on raw tensors (no checks beyond the library's own)."""
+            out, last_state, ckpt, stream=None, zoh: bool = False):
+    """Direct C-ABI call on raw tensors (no checks beyond the library's own).
+    zoh selects the zero-order-hold B̄ (ssm_selective_scan_fwd_ex)."""
+    if zoh:
+        o = _opts(delta_softplus, True)
+        _check(load_library().ssm_selective_scan_fwd_ex(
+            ctypes.byref(shape), ctypes.byref(o), _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C),
+            _ptr(D), _ptr(z), _ptr(delta_bias), _ptr(out), _ptr(last_state), _ptr(ckpt),
+            _stream_ptr(stream)))
+        return
     _check(load_library().ssm_selective_scan_fwd(
         ctypes.byref(shape), _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
         _ptr(delta_bias), int(bool(delta_softplus)), _ptr(out), _ptr(last_state), _ptr(ckpt),
@@ -133,8 +159,17 @@ def fwd_raw(shape: Shape, u, delta, A, B, C, D, z, delta_bias, delta_softplus: b
 
 
 def bwd_raw(shape: Shape, u, delta, A, B, C, D, z, delta_bias, delta_softplus: bool, dout,
-            ckpt, du, ddelta, dA, dB, dC, dD, dz, ddelta_bias, scratch, stream=None):
+            ckpt, du, ddelta, dA, dB, dC, dD, dz, ddelta_bias, scratch, stream=None,
+            zoh: bool = False):
     nbytes = 0 if scratch is None else scratch.numel() * scratch.element_size()
+    if zoh:
+        o = _opts(delta_softplus, True)
+        _check(load_library().ssm_selective_scan_bwd_ex(
+            ctypes.byref(shape), ctypes.byref(o), _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C),
+            _ptr(D), _ptr(z), _ptr(delta_bias), _ptr(dout), _ptr(ckpt), _ptr(du), _ptr(ddelta),
+            _ptr(dA), _ptr(dB), _ptr(dC), _ptr(dD), _ptr(dz), _ptr(ddelta_bias), _ptr(scratch),
+            ctypes.c_size_t(nbytes), _stream_ptr(stream)))
+        return
     _check(load_library().ssm_selective_scan_bwd(
         ctypes.byref(shape), _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
         _ptr(delta_bias), int(bool(delta_softplus)), _ptr(dout), _ptr(ckpt), _ptr(du),
@@ -154,9 +189,15 @@ def bwd_noalloc_raw(shape: Shape, u, delta, A, B, C, D, z, delta_bias, delta_sof
 
 
 def state_update_raw(shape: Shape, state, u, delta, A, B, C, D, z, delta_bias,
-                     delta_softplus: bool, out, stream=None):
-    """Direct call of ssm_selective_state_update (one decoding step, state
+                     delta_softplus: bool, out, stream=None, zoh: bool = False):
+    """Direct call of ssm_selective_state_update(_ex) (one decoding step, state
     updated in place)."""
+    if zoh:
+        o = _opts(delta_softplus, True)
+        _check(load_library().ssm_selective_state_update_ex(
+            ctypes.byref(shape), ctypes.byref(o), _ptr(state), _ptr(u), _ptr(delta), _ptr(A),
+            _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias), _ptr(out), _stream_ptr(stream)))
+        return
     _check(load_library().ssm_selective_state_update(
         ctypes.byref(shape), _ptr(state), _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
         _ptr(z), _ptr(delta_bias), int(bool(delta_softplus)), _ptr(out), _stream_ptr(stream)))
@@ -175,7 +216,7 @@ def _need(t, name, dtype=None, cuda=True):
 
 def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None,
                        delta_softplus: bool = True, return_last_state: bool = False,
-                       return_ckpt: bool = False, out=None, stream=None):
+                       return_ckpt: bool = False, out=None, stream=None, zoh: bool = False):
     """Forward selective scan.  u, delta, z, B, C share one io dtype (float32 or
     bfloat16); A, D, delta_bias are float32.  Returns (out, last_state, ckpt)
     with the last two None unless requested."""
@@ -191,12 +232,12 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None,
                         dtype=torch.float32) if return_last_state else None)
     ck = (torch.empty(ckpt_numel(shape), device=u.device, dtype=torch.float32)
           if return_ckpt else None)
-    fwd_raw(shape, u, delta, A, B, C, D, z, delta_bias, delta_softplus, out, last, ck, stream)
+    fwd_raw(shape, u, delta, A, B, C, D, z, delta_bias, delta_softplus, out, last, ck, stream, zoh)
     return out, last, ck
 
 
 def selective_state_update(state, u, delta, A, B, C, D=None, z=None, delta_bias=None,
-                           delta_softplus: bool = True, out=None, stream=None):
+                           delta_softplus: bool = True, out=None, stream=None, zoh: bool = False):
     """One decoding step: advances `state` ([batch, dim, dstate] float32) in
     place by one token and returns out [batch, dim].  u, delta, z are
     [batch, dim] and B, C [batch, dstate] in one io dtype; A, D, delta_bias
@@ -211,15 +252,16 @@ def selective_state_update(state, u, delta, A, B, C, D=None, z=None, delta_bias=
     shape = make_shape(u.shape[0], u.shape[1], 1, A.shape[1], io)
     if out is None:
         out = torch.empty_like(u)
-    state_update_raw(shape, state, u, delta, A, B, C, D, z, delta_bias, delta_softplus, out, stream)
+    state_update_raw(shape, state, u, delta, A, B, C, D, z, delta_bias, delta_softplus, out, stream,
+                     zoh)
     return out
 
 
 def selective_scan_bwd(u, delta, A, B, C, D, z, delta_bias, delta_softplus: bool, dout,
-                       ckpt=None, stream=None):
+                       ckpt=None, stream=None, zoh: bool = False):
     """Backward selective scan; returns a dict of float32 gradients (du, ddelta,
     dA, dB, dC and, for the optional inputs that were given, dD, dz,
-    ddelta_bias)."""
+    ddelta_bias).  zoh must match the forward that wrote `ckpt`."""
     io = u.dtype
     for t, n in ((u, "u"), (delta, "delta"), (B, "B"), (C, "C"), (z, "z"), (dout, "dout")):
         _need(t, n, io)
@@ -237,5 +279,5 @@ def selective_scan_bwd(u, delta, A, B, C, D, z, delta_bias, delta_softplus: bool
     scratch = torch.empty(max(1, nscratch // 4), **f32) if nscratch else None
     bwd_raw(shape, u, delta, A, B, C, D, z, delta_bias, delta_softplus, dout, ckpt,
             g["du"], g["ddelta"], g["dA"], g["dB"], g["dC"], g["dD"], g["dz"],
-            g["ddelta_bias"], scratch, stream)
+            g["ddelta_bias"], scratch, stream, zoh)
     return {k: v for k, v in g.items() if v is not None}
