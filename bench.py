@@ -152,6 +152,18 @@ def max_over_ranks(x: float, world: int) -> float:
     return float(t.item())
 
 
+def rank_seed(seed: int, rank: int) -> int:
+    """Seed of a rank's own batch: every rank draws different inputs of the same
+    shape (weak scaling, no shared data)."""
+    return seed + 7919 * rank
+
+
+def aggregate_rate(world: int, steps: int, units_per_step: int, t_dev_s: float) -> float:
+    """Whole-job throughput: the units all ranks processed over the slowest
+    rank's device time (max over ranks)."""
+    return world * steps * units_per_step / max_over_ranks(t_dev_s, world)
+
+
 def cpu_oracle_rate(w, inp, budget_s: float, nthreads: int = 0):
     """Times the fp64 oracle on whole-batch channel slices until about
     `budget_s` seconds of wall time are spent.  Returns (elem/s, threads, desc)."""
@@ -238,7 +250,7 @@ def run_ours(args, world, rank, local):
         w = w.replace(seqlen=args.seqlen, name=f"{w.name}_L{args.seqlen}")
     dev = torch.device("cuda", local)
     # every rank processes its own batch of the same shape (weak scaling)
-    w_rank = w.replace(seed=w.seed + 7919 * rank)
+    w_rank = w.replace(seed=rank_seed(w.seed, rank))
     fwdbwd = w.name.startswith("mamba130m_layer_fwdbwd")
     inp = generate(w_rank, with_dout=fwdbwd)
     dv = to_torch(inp, w_rank, dev)
@@ -389,7 +401,7 @@ def run_decode(args, world, rank, local):
     from selective_state_space_50_b200 import ssm_scan
     from selective_state_space_50_b200.workloads import Workload, generate, to_torch
 
-    w = Workload("decode_step_2p8b", 64, 1, 5120, 16, "bf16", seed=1005 + 7919 * rank,
+    w = Workload("decode_step_2p8b", 64, 1, 5120, 16, "bf16", seed=rank_seed(1005, rank),
                  D_dist="u0.5_1.5")
     dev = torch.device("cuda", local)
     inp = generate(w)

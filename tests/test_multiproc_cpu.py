@@ -1,0 +1,80 @@
+"""The multi-rank (N > 1) host path of bench.py on CPU: two processes with the
+gloo backend, rendezvous on 127.0.0.1.  The GPU machine runs one GPU per call, so
+these are the tests of the rank logic."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out_q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), WORLD_SIZE=str(world),
+                      RANK=str(rank), LOCAL_RANK=str(rank))
+    import torch.distributed as dist
+
+    class A:
+        gpus = world
+    w, r, _ = bench.dist_setup(A())
+    try:
+        bench.barrier(w)
+        m = bench.max_over_ranks(1.5 + r, w)
+        # rank r "took" 1 + r seconds for 10 steps of 100 units each
+        rate = bench.aggregate_rate(w, 10, 100, 1.0 + r)
+        out_q.put((r, m, rate))
+        bench.barrier(w)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_and_aggregate_rate_gloo():
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(world))
+    for r, m, rate in res:
+        assert m == 2.5                             # max over ranks, seen by every rank
+        assert rate == pytest.approx(2 * 10 * 100 / 2.0)   # all units over the slowest rank
+
+
+def test_rank_seeds_differ():
+    seeds = {bench.rank_seed(1001, r) for r in range(8)}
+    assert len(seeds) == 8
+
+
+def test_reference_arm_under_torchrun():
+    """`--impl reference` launched as the driver launches multi-GPU runs: rank 0
+    alone prints one JSON line, the other rank exits 0 without work."""
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(_free_port()),
+           os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+           "--steps", "1", "--warmup", "0"]
+    r = subprocess.run(cmd, env=env, capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
+    assert d["e2e"]["h2d_bytes_per_step"] == 0
