@@ -283,6 +283,16 @@ ssm_status_t ssm_selective_state_update_ex(const ssm_shape_t *shape, const ssm_o
  */
 ssm_status_t ssm_device_error_status(void *stream);
 
+/*
+ * Diagnostic: launches on `stream` a one-warp kernel whose bounded wait (on a
+ * shared-memory barrier that nothing completes) gives up after about 1 ms of
+ * SM clock and sets the device error word, exactly as a stalled copy would.
+ * The next ssm_device_error_status then returns SSM_ERR_TIMEOUT (and clears
+ * the word).  Nothing faults or hangs; the stream stays usable.  The pages
+ * have no counterpart: this exists to test the library's failure reporting.
+ */
+ssm_status_t ssm_selftest_wait_timeout(void *stream);
+
 #ifdef __cplusplus
 }
 #endif

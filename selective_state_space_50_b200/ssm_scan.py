@@ -27,7 +27,7 @@ EXPORTS = ("ssm_version", "ssm_last_error_string", "ssm_selective_scan_ckpt_byte
            "ssm_selective_scan_bwd", "ssm_device_error_status",
            "ssm_selective_scan_bwd_noalloc", "ssm_selective_state_update",
            "ssm_selective_scan_fwd_ex", "ssm_selective_scan_bwd_ex",
-           "ssm_selective_state_update_ex")
+           "ssm_selective_state_update_ex", "ssm_selftest_wait_timeout")
 SSM_DISC_DELTA_B, SSM_DISC_ZOH = 0, 1
 NOALLOC_SCRATCH_BYTES = 32 << 20  # SSM_NOALLOC_SCRATCH_BYTES in include/ssm_scan.h
 
@@ -88,6 +88,8 @@ def load_library(path: str = LIB_PATH):
     lib.ssm_selective_scan_bwd_ex.restype = i
     lib.ssm_selective_state_update_ex.argtypes = [sp, op] + [vp] * 11
     lib.ssm_selective_state_update_ex.restype = i
+    lib.ssm_selftest_wait_timeout.argtypes = [vp]
+    lib.ssm_selftest_wait_timeout.restype = i
     _lib = lib
     return lib
 
