@@ -132,3 +132,52 @@ def bwd_workload(inputs: Dict[str, np.ndarray], w, nthreads: int = 0):
                inputs["z_f64"] if w.has_z else None,
                inputs["delta_bias_f64"] if w.has_bias else None, w.softplus,
                inputs["dout_f64"], nthreads=nthreads)
+
+
+# ------------------------------------------------------------------ selection projections
+# The selection mechanism makes B, C and the step size functions of the input
+# (Mamba paper review on booiljung.github.io, "3.2 선택적 스캔(Selective Scan)
+# 알고리즘", §1.2: B_t = Linear_N(x_t), C_t = Linear_N(x_t),
+# Δ_t = Softplus(Parameter + Linear_1(x_t)); honbul.tistory.com, "Mamba" §2:
+# B_t = s_B(x_t), C_t = s_C(x_t), Δ_t = softplus(Δ + s_Δ(x_t))).  The step-size
+# projection is taken as a rank-R factorisation Linear_D(Linear_R(x)): R = 1
+# with an all-ones up-projection is the pages' Broadcast_D(Linear_1(x)).  The
+# Parameter (the per-channel bias) and the softplus stay in the scan.
+
+def bf16_round(v) -> np.ndarray:
+    """Round-to-nearest-even to bfloat16 of float64 values (through float32,
+    as an fp32 accumulator would be stored), returned as float64."""
+    f = np.ascontiguousarray(v, dtype=np.float64).astype(np.float32)
+    bits = f.view(np.uint32).astype(np.uint64)
+    lsb = (bits >> np.uint64(16)) & np.uint64(1)
+    r = ((bits + np.uint64(0x7FFF) + lsb) >> np.uint64(16)) << np.uint64(16)
+    out = r.astype(np.uint32).view(np.float32).astype(np.float64)
+    # NaN/Inf inputs keep their class (the rounding above would not carry them)
+    special = ~np.isfinite(f)
+    out[special] = f[special]
+    return out
+
+
+def projections(x, W_x, W_dt, dt_rank: int, dstate: int, store_low_bf16: bool = True):
+    """x [b, D, L]; W_x [R + 2N, D]; W_dt [D, R].
+
+    For every batch row and step t: xdbl_t = W_x x_t (one Linear over the
+    channels), split into the low-rank step-size input dt_low_t = xdbl_t[0:R],
+    B_t = xdbl_t[R:R+N] and C_t = xdbl_t[R+N:R+2N]; then delta_t = W_dt dt_low_t.
+    dt_low is an intermediate stored in bfloat16 before the second Linear
+    (store_low_bf16); the second product uses those stored values.
+
+    Returns float64 (dt_low [b,R,L], delta [b,D,L], B [b,N,L], C [b,N,L]),
+    unrounded apart from the stored intermediate."""
+    x, W_x, W_dt = map(_f64, (x, W_x, W_dt))
+    batch, dim, L = x.shape
+    R, N = int(dt_rank), int(dstate)
+    assert W_x.shape == (R + 2 * N, dim) and W_dt.shape == (dim, R)
+    xdbl = np.matmul(W_x[None, :, :], x)                 # [b, R+2N, L]
+    dt_low = xdbl[:, :R]
+    B = xdbl[:, R:R + N]
+    C = xdbl[:, R + N:]
+    low = bf16_round(dt_low) if store_low_bf16 else dt_low
+    delta = np.matmul(W_dt[None, :, :], low)             # [b, D, L]
+    return (np.ascontiguousarray(dt_low), np.ascontiguousarray(delta),
+            np.ascontiguousarray(B), np.ascontiguousarray(C))

@@ -37,7 +37,7 @@ _M2 = np.uint64(0x94D049BB133111EB)
 
 # Stream ids: one independent counter stream per tensor.
 STREAMS = {"delta_bias": 1, "D": 2, "A": 3, "u": 4, "delta": 5, "z": 6,
-           "B": 7, "C": 8, "dout": 9, "delta0": 10}
+           "B": 7, "C": 8, "dout": 9, "delta0": 10, "x": 11, "W_x": 12, "W_dt": 13}
 
 _CHUNK = 1 << 22  # elements generated per numpy pass (bounds host memory)
 
@@ -272,3 +272,29 @@ def to_torch(inputs: Dict[str, np.ndarray], w: Workload, device):
     if not w.has_bias:
         d["delta_bias"] = None
     return d
+
+
+# ---------------------------------------------------------------- projections
+
+def generate_projection(batch: int, dim: int, seqlen: int, dstate: int, dt_rank: int,
+                        seed: int) -> Dict[str, np.ndarray]:
+    """Inputs of the selection projections, all bf16 (uint16 bit patterns,
+    with the exact values under name + "_f64"):
+
+        x    [batch, dim, seqlen] ~ N(0, 1)          (the scan's input u)
+        W_x  [dt_rank + 2 dstate, dim] ~ N(0, 1/dim)  (rows: dt_low, B, C)
+        W_dt [dim, dt_rank] ~ N(0, 1/dt_rank)
+
+    The weight scales keep every projected value near unit variance, like
+    the scan's own synthetic delta, B and C."""
+    out: Dict[str, np.ndarray] = {}
+    M = dt_rank + 2 * dstate
+    draws = {
+        "x": normal(seed, STREAMS["x"], batch * dim * seqlen).reshape(batch, dim, seqlen),
+        "W_x": normal(seed, STREAMS["W_x"], M * dim, 1.0 / math.sqrt(dim)).reshape(M, dim),
+        "W_dt": normal(seed, STREAMS["W_dt"], dim * dt_rank,
+                       1.0 / math.sqrt(dt_rank)).reshape(dim, dt_rank),
+    }
+    for name, x in draws.items():
+        out[name], out[name + "_f64"] = _cast(x, "bf16")
+    return out
