@@ -133,7 +133,9 @@ __device__ __forceinline__ float4 f4add(float4 a, float4 b) {
     return make_float4(lo.x, lo.y, hi.x, hi.y);
 }
 
-template <typename T, int NWC, int STAGES, bool HZ, bool SP>
+// ALN: the channel count is a multiple of 8 and CTAs and passes start on
+// multiples of 8 rows, so that no warp's 8 channels span two batch rows.
+template <typename T, int NWC, int STAGES, bool HZ, bool SP, bool ALN>
 __global__ void __launch_bounds__((NWC + 1) * 32, 1)
 bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constant__ CUtensorMap m_u,
                const __grid_constant__ CUtensorMap m_z, const __grid_constant__ CUtensorMap m_g,
@@ -155,8 +157,9 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int G = gridDim.x;
-    const int r0 = (int)((long long)blockIdx.x * p.P / G);
-    const int r1 = (int)((long long)(blockIdx.x + 1) * p.P / G);
+    constexpr int RU = ALN ? CPW : 1;   // rows are split in units of RU
+    const int r0 = RU * (int)((long long)blockIdx.x * (p.P / RU) / G);
+    const int r1 = RU * (int)((long long)(blockIdx.x + 1) * (p.P / RU) / G);
     const int R = r1 - r0;
     const int npass = (R + p.rows_max - 1) / p.rows_max;
     const int ntiles = (p.L + TT - 1) / TT;
@@ -178,8 +181,8 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
     __syncthreads();
 
     auto pass_rows = [&](int q, int &q0, int &q1) {
-        q0 = r0 + (int)((long long)q * R / npass);
-        q1 = r0 + (int)((long long)(q + 1) * R / npass);
+        q0 = r0 + RU * (int)((long long)q * (R / RU) / npass);
+        q1 = r0 + RU * (int)((long long)(q + 1) * (R / RU) / npass);
     };
     // batch rows [b_lo, b_lo + nb) touched by pass q
     auto pass_batches = [&](int q, int &b_lo, int &nb) {
@@ -334,7 +337,7 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
             bsel = live ? row / p.dim - q0 / p.dim : 0;
             const unsigned lmask = __ballot_sync(0xffffffffu, live) & 0xffu;
             b1mask = __ballot_sync(0xffffffffu, bsel == 1) & 0xffu;
-            straddle = b1mask != 0 && b1mask != lmask;
+            straddle = !ALN && b1mask != 0 && b1mask != lmask;
             wb = b1mask != 0 ? 1 : 0;
 #pragma unroll
             for (int j = 0; j < NS; ++j) {
@@ -421,7 +424,7 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                 const float *src = wX + g * CPW * XS + c * 4;
                 const int n = g * NS + (c >> 1), tb = tw + (c & 1) * 4;
                 float *dst = dbuf + (which * 2 * N + n) * TT;
-                if (!straddle) {
+                if (ALN || !straddle) {
                     float4 s0 = *reinterpret_cast<const float4 *>(src);
 #pragma unroll
                     for (int cc = 1; cc < CPW; ++cc) s0 = f4add(s0, *reinterpret_cast<const float4 *>(src + cc * XS));
@@ -620,11 +623,11 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
 // ------------------------------------------------------------------ host side
 
 
-template <typename T, int NWC, int STAGES, bool HZ, bool SP>
+template <typename T, int NWC, int STAGES, bool HZ, bool SP, bool ALN>
 cudaError_t launch_bwd_tma_cfg(const BwdParams &bp, int rows_max, cudaStream_t stream) {
     using Ly = BwdLayout<T, NWC, STAGES>;
     const int P = bp.batch * bp.dim;
-    const int grid = std::min(device_sm_count(), P);
+    const int grid = std::min(device_sm_count(), ALN ? P / Ly::CPW : P);
     const bool bf16 = sizeof(T) == 2;
     CUtensorMap md, mu, mz, mg, mB, mC;
     const uint32_t bc_box = Ly::PW / sizeof(T);
@@ -643,7 +646,7 @@ cudaError_t launch_bwd_tma_cfg(const BwdParams &bp, int rows_max, cudaStream_t s
     p.softplus = bp.softplus; p.has_z = bp.z != nullptr; p.rows_max = rows_max;
     p.err = device_error_word();
     if (!p.err) return cudaErrorInvalidDevice;
-    auto kern = bwd_tma_kernel<T, NWC, STAGES, HZ, SP>;
+    auto kern = bwd_tma_kernel<T, NWC, STAGES, HZ, SP, ALN>;
     static bool attr_done = false;
     if (!attr_done) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Ly::kAlloc);
@@ -654,14 +657,28 @@ cudaError_t launch_bwd_tma_cfg(const BwdParams &bp, int rows_max, cudaStream_t s
     return cudaGetLastError();
 }
 
-// The gate and the softplus are compile-time switches of the kernel.
-template <typename T, int NWC>
+// Depth of the ring of input tiles.
+#ifndef SSM_BWD_STAGES
+#define SSM_BWD_STAGES 2
+#endif
+constexpr int kBwdStages = SSM_BWD_STAGES;
+
+// The gate, the softplus and the 8-row alignment are compile-time switches
+// of the kernel.
+template <typename T, int NWC, bool ALN>
 cudaError_t launch_bwd_tma_flags(const BwdParams &bp, int rows_max, cudaStream_t stream) {
     const bool hz = bp.z != nullptr, sp = bp.softplus != 0;
-    if (hz && sp) return launch_bwd_tma_cfg<T, NWC, 2, true, true>(bp, rows_max, stream);
-    if (hz) return launch_bwd_tma_cfg<T, NWC, 2, true, false>(bp, rows_max, stream);
-    if (sp) return launch_bwd_tma_cfg<T, NWC, 2, false, true>(bp, rows_max, stream);
-    return launch_bwd_tma_cfg<T, NWC, 2, false, false>(bp, rows_max, stream);
+    constexpr int S = kBwdStages;
+    if (hz && sp) return launch_bwd_tma_cfg<T, NWC, S, true, true, ALN>(bp, rows_max, stream);
+    if (hz) return launch_bwd_tma_cfg<T, NWC, S, true, false, ALN>(bp, rows_max, stream);
+    if (sp) return launch_bwd_tma_cfg<T, NWC, S, false, true, ALN>(bp, rows_max, stream);
+    return launch_bwd_tma_cfg<T, NWC, S, false, false, ALN>(bp, rows_max, stream);
+}
+
+template <typename T, int NWC>
+cudaError_t launch_bwd_tma_aln(const BwdParams &bp, int rows_max, bool aln, cudaStream_t stream) {
+    return aln ? launch_bwd_tma_flags<T, NWC, true>(bp, rows_max, stream)
+               : launch_bwd_tma_flags<T, NWC, false>(bp, rows_max, stream);
 }
 
 bool aligned_to(const void *ptr, uintptr_t a) { return (reinterpret_cast<uintptr_t>(ptr) % a) == 0; }
@@ -690,13 +707,18 @@ bool try_launch_bwd_tma(const BwdParams &bp, cudaStream_t stream, cudaError_t *e
     const long long P = (long long)bp.batch * bp.dim;
     const int sms = device_sm_count();
     if (P < sms) return false;
-    const long long cap = (bp.io_bf16 ? kBwdWarpsBf16 : kBwdWarpsF32) * 8;
-    const long long R = (P + sms - 1) / sms;
+    // rows are split over the CTAs in units of 8 when the channel count
+    // allows it (one unit per consumer warp), else one by one
+    const bool aln = bp.dim % 8 == 0;
+    const long long unit = aln ? 8 : 1;
+    const long long cap = (bp.io_bf16 ? kBwdWarpsBf16 : kBwdWarpsF32) * 8 / unit;
+    const long long U = P / unit;
+    const long long R = (U + sms - 1) / sms;
     const long long npass = (R + cap - 1) / cap;
-    const long long rows_max = (R + npass - 1) / npass;
+    const long long rows_max = unit * ((R + npass - 1) / npass);
     if (rows_max > bp.dim) return false;   // a pass spans at most two batch rows
-    *err = bp.io_bf16 ? launch_bwd_tma_flags<__nv_bfloat16, kBwdWarpsBf16>(bp, (int)rows_max, stream)
-                      : launch_bwd_tma_flags<float, kBwdWarpsF32>(bp, (int)rows_max, stream);
+    *err = bp.io_bf16 ? launch_bwd_tma_aln<__nv_bfloat16, kBwdWarpsBf16>(bp, (int)rows_max, aln, stream)
+                      : launch_bwd_tma_aln<float, kBwdWarpsF32>(bp, (int)rows_max, aln, stream);
     return true;
 }
 
