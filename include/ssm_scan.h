@@ -293,6 +293,48 @@ ssm_status_t ssm_device_error_status(void *stream);
  */
 ssm_status_t ssm_selftest_wait_timeout(void *stream);
 
+/*
+ * Selection projections: the per-token Linear layers that make the scan's
+ * step size, B and C functions of its input x (= u of the scan).
+ * booiljung.github.io, "3.2 선택적 스캔(Selective Scan) 알고리즘과 정보의 압축
+ * 및 선별", §1.2: B_t = Linear_N(x_t), C_t = Linear_N(x_t),
+ * Δ_t = Softplus(Parameter + Linear_1(x_t)); honbul.tistory.com, "Mamba" §2
+ * (s_B, s_C, s_Δ).  The step-size projection is taken as the rank-R
+ * factorisation Linear_D(Linear_R(x)); the pages' broadcast Linear_1 is
+ * R = 1 with an all-ones up-projection, which this call expresses with
+ * dt_rank = 8 and zero weights in the seven extra rows and columns.  The
+ * Parameter (delta_bias) and the softplus are applied by the scan.
+ *
+ * For every batch row b and step t, with M1 = dt_rank + 2 * dstate:
+ *   xdbl_t  = W_x · x[b, :, t]                 (M1 values, fp32 accumulation)
+ *   dt_low[b, r, t] = xdbl_t[r]                r < dt_rank
+ *   B[b, n, t]      = xdbl_t[dt_rank + n]
+ *   C[b, n, t]      = xdbl_t[dt_rank + dstate + n]
+ *   delta[b, d, t]  = Σ_r W_dt[d, r] dt_low[b, r, t]   (on the bf16-stored dt_low)
+ * Every output is rounded to bfloat16 (nearest even) from fp32.
+ *
+ * Layouts (row-major, all bfloat16, all device memory owned by the caller):
+ *   x       [batch][dim][seqlen]          W_x   [M1][dim]
+ *   W_dt    [dim][dt_rank]                dt_low [batch][dt_rank][seqlen]
+ *   delta   [batch][dim][seqlen]          B, C  [batch][dstate][seqlen]
+ * B, C and delta are exactly the scan's inputs of the same names; dt_low is
+ * an intermediate the caller provides the memory for.  Outputs must not
+ * overlap the inputs or each other.
+ *
+ * Requirements: every pointer 16-byte aligned; seqlen, dim and dt_rank
+ * multiples of 8; 1 <= dstate <= 64; batch <= 65535; io_dtype SSM_BF16
+ * (shape->dstate and shape->io_dtype are read from `shape`, `dt_rank` is
+ * separate).  Runs on the tensor cores (tcgen05, fp32 accumulators in tensor
+ * memory) as two launches on `stream`.
+ * Errors: SSM_ERR_INVALID_ARG (NULL, misaligned, host or overlapping
+ * pointers, sizes not multiples of 8), SSM_ERR_UNSUPPORTED (io dtype, dstate,
+ * batch, no tensor-map support in the driver), SSM_ERR_CUDA.
+ */
+ssm_status_t ssm_selection_projections(const ssm_shape_t *shape, int dt_rank,
+                                       const void *x, const void *W_x, const void *W_dt,
+                                       void *dt_low, void *delta, void *B, void *C,
+                                       void *stream);
+
 #ifdef __cplusplus
 }
 #endif

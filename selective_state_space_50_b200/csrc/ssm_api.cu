@@ -346,6 +346,47 @@ ssm_status_t ssm_selective_state_update(const ssm_shape_t *shape, float *state, 
                                          out, stream);
 }
 
+ssm_status_t ssm_selection_projections(const ssm_shape_t *shape, int dt_rank, const void *x,
+                                       const void *W_x, const void *W_dt, void *dt_low, void *delta,
+                                       void *B, void *C, void *stream) {
+    if (!shape) return fail(SSM_ERR_INVALID_ARG, "shape is NULL");
+    const ssm_shape_t &s = *shape;
+    if (s.batch < 1 || s.dim < 1 || s.seqlen < 1 || s.dstate < 1 || dt_rank < 1)
+        return fail(SSM_ERR_INVALID_ARG, "batch, dim, seqlen, dstate, dt_rank must be >= 1");
+    if (s.io_dtype != SSM_BF16)
+        return fail(SSM_ERR_UNSUPPORTED, "the projections take bfloat16 only");
+    if (s.seqlen % 8 || s.dim % 8 || dt_rank % 8)
+        return fail(SSM_ERR_INVALID_ARG, "seqlen, dim and dt_rank must be multiples of 8 (got %d, %d, %d)",
+                    s.seqlen, s.dim, dt_rank);
+    if (s.dstate > 64) return fail(SSM_ERR_UNSUPPORTED, "dstate %d > 64", s.dstate);
+    if (s.batch > 65535) return fail(SSM_ERR_UNSUPPORTED, "batch %d > 65535", s.batch);
+    const long long M1 = dt_rank + 2LL * s.dstate;
+    if ((long long)s.batch * s.dim * s.seqlen >= (1LL << 31) ||
+        (long long)s.batch * M1 * s.seqlen >= (1LL << 31) || (long long)s.dim * M1 >= (1LL << 31))
+        return fail(SSM_ERR_UNSUPPORTED, "tensor sizes must be < 2^31 elements");
+    const void *ptrs[] = {x, W_x, W_dt, dt_low, delta, B, C};
+    const char *names[] = {"x", "W_x", "W_dt", "dt_low", "delta", "B", "C"};
+    for (int i = 0; i < 7; ++i) SSM_TRY(check_ptr(ptrs[i], names[i], 16, true));
+    const size_t bytes[] = {
+        (size_t)s.batch * s.dim * s.seqlen * 2, (size_t)M1 * s.dim * 2, (size_t)s.dim * dt_rank * 2,
+        (size_t)s.batch * dt_rank * s.seqlen * 2, (size_t)s.batch * s.dim * s.seqlen * 2,
+        (size_t)s.batch * s.dstate * s.seqlen * 2, (size_t)s.batch * s.dstate * s.seqlen * 2};
+    for (int i = 3; i < 7; ++i)          // every output against every other tensor
+        for (int j = 0; j < 7; ++j) {
+            if (i == j) continue;
+            const uintptr_t a0 = (uintptr_t)ptrs[i], a1 = a0 + bytes[i];
+            const uintptr_t b0 = (uintptr_t)ptrs[j], b1 = b0 + bytes[j];
+            if (a0 < b1 && b0 < a1)
+                return fail(SSM_ERR_INVALID_ARG, "%s overlaps %s", names[i], names[j]);
+        }
+    if (!ssm::tma_available()) return fail(SSM_ERR_UNSUPPORTED, "the driver has no tensor-map encoder");
+    const ssm::ProjShape ps{s.batch, s.dim, s.seqlen, s.dstate, dt_rank};
+    cudaError_t e = ssm::launch_projections(ps, x, W_x, W_dt, dt_low, delta, B, C,
+                                            static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "ssm_selection_projections launch");
+    return ok();
+}
+
 ssm_status_t ssm_device_error_status(void *stream) {
     int v = 0;
     cudaError_t e = ssm::read_and_clear_device_error(&v, static_cast<cudaStream_t>(stream));

@@ -59,6 +59,14 @@ struct StepParams {
     bool vec_ok;                   // state, A, B, C 16-byte aligned (vector access)
 };
 
+// Selection projections (ssm_proj.cu): x_proj then dt_proj on the tensor
+// cores, bf16 in and out.
+struct ProjShape {
+    int batch, dim, seqlen, dstate, dt_rank;
+};
+cudaError_t launch_projections(const ProjShape &s, const void *x, const void *W_x, const void *W_dt,
+                               void *dt_low, void *delta, void *B, void *C, cudaStream_t stream);
+
 // Single-step recurrent update (ssm_step.cu).
 cudaError_t launch_state_update(const StepParams &p, cudaStream_t stream);
 
@@ -88,6 +96,11 @@ cudaError_t launch_bwd(const BwdParams &p, cudaStream_t stream);
 bool tma_available();
 bool make_tma_map_2d(CUtensorMap *m, const void *base, bool bf16, uint64_t rows, uint64_t cols,
                      uint32_t box_cols, uint32_t box_rows, bool swizzle128);
+// make_tma_map_bf16_3d: a bf16 tensor of extents {d0 (contiguous), d1, d2},
+// tiles of {box0, box1, 1} with the 128-byte swizzle; out-of-range elements
+// of a tile read 0.
+bool make_tma_map_bf16_3d(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64_t d2,
+                          uint32_t box0, uint32_t box1);
 int device_sm_count();
 // Launches the TMA-fed persistent backward when it applies (dstate 16, 16-byte
 // aligned rows and checkpoints, at least one channel row per SM); returns

@@ -27,7 +27,8 @@ EXPORTS = ("ssm_version", "ssm_last_error_string", "ssm_selective_scan_ckpt_byte
            "ssm_selective_scan_bwd", "ssm_device_error_status",
            "ssm_selective_scan_bwd_noalloc", "ssm_selective_state_update",
            "ssm_selective_scan_fwd_ex", "ssm_selective_scan_bwd_ex",
-           "ssm_selective_state_update_ex", "ssm_selftest_wait_timeout")
+           "ssm_selective_state_update_ex", "ssm_selftest_wait_timeout",
+           "ssm_selection_projections")
 SSM_DISC_DELTA_B, SSM_DISC_ZOH = 0, 1
 NOALLOC_SCRATCH_BYTES = 32 << 20  # SSM_NOALLOC_SCRATCH_BYTES in include/ssm_scan.h
 
@@ -90,6 +91,8 @@ def load_library(path: str = LIB_PATH):
     lib.ssm_selective_state_update_ex.restype = i
     lib.ssm_selftest_wait_timeout.argtypes = [vp]
     lib.ssm_selftest_wait_timeout.restype = i
+    lib.ssm_selection_projections.argtypes = [sp, i] + [vp] * 8
+    lib.ssm_selection_projections.restype = i
     _lib = lib
     return lib
 
@@ -205,6 +208,13 @@ def state_update_raw(shape: Shape, state, u, delta, A, B, C, D, z, delta_bias,
         _ptr(z), _ptr(delta_bias), int(bool(delta_softplus)), _ptr(out), _stream_ptr(stream)))
 
 
+def projections_raw(shape: Shape, dt_rank: int, x, W_x, W_dt, dt_low, delta, B, C, stream=None):
+    """Direct call of ssm_selection_projections (x_proj then dt_proj)."""
+    _check(load_library().ssm_selection_projections(
+        ctypes.byref(shape), int(dt_rank), _ptr(x), _ptr(W_x), _ptr(W_dt), _ptr(dt_low),
+        _ptr(delta), _ptr(B), _ptr(C), _stream_ptr(stream)))
+
+
 def _need(t, name, dtype=None, cuda=True):
     if t is None:
         return
@@ -283,3 +293,26 @@ def selective_scan_bwd(u, delta, A, B, C, D, z, delta_bias, delta_softplus: bool
             g["du"], g["ddelta"], g["dA"], g["dB"], g["dC"], g["dD"], g["dz"],
             g["ddelta_bias"], scratch, stream, zoh)
     return {k: v for k, v in g.items() if v is not None}
+
+
+def selection_projections(x, W_x, W_dt, dstate: int, stream=None):
+    """The selection projections in front of the scan: x [batch, dim, L],
+    W_x [dt_rank + 2 dstate, dim], W_dt [dim, dt_rank], all bfloat16.
+    Returns (delta [batch, dim, L], B [batch, dstate, L], C [batch, dstate, L],
+    dt_low [batch, dt_rank, L]); delta, B and C are the scan's inputs."""
+    for t, n in ((x, "x"), (W_x, "W_x"), (W_dt, "W_dt")):
+        _need(t, n, torch.bfloat16)
+    if x.dim() != 3 or W_x.dim() != 2 or W_dt.dim() != 2:
+        raise ValueError("x must be [batch, dim, L], W_x [M, dim] and W_dt [dim, dt_rank]")
+    batch, dim, L = x.shape
+    dt_rank = W_dt.shape[1]
+    if W_dt.shape[0] != dim or tuple(W_x.shape) != (dt_rank + 2 * dstate, dim):
+        raise ValueError("W_x must be [dt_rank + 2 dstate, dim] and W_dt [dim, dt_rank]")
+    shape = make_shape(batch, dim, L, dstate, SSM_BF16)
+    kw = dict(device=x.device, dtype=torch.bfloat16)
+    dt_low = torch.empty(batch, dt_rank, L, **kw)
+    delta = torch.empty(batch, dim, L, **kw)
+    B = torch.empty(batch, dstate, L, **kw)
+    C = torch.empty(batch, dstate, L, **kw)
+    projections_raw(shape, dt_rank, x, W_x, W_dt, dt_low, delta, B, C, stream)
+    return delta, B, C, dt_low
