@@ -59,13 +59,25 @@ def algorithmic_bytes(w, io_bytes, with_last_state=True, backward=False):
     if with_last_state:
         n += w.batch * w.dim * w.dstate * 4
     if backward:
-        nck = -(-w.seqlen // 64)
-        ck = w.batch * w.dim * nck * w.dstate * 4
-        n += ck                                         # forward writes checkpoints
-        n += e * io_bytes * 4 + 2 * bc * io_bytes + ck  # u, delta, z, dout, B, C, ckpt read
+        # the checkpoints (8 bytes per element each way at N = 16) are this
+        # design's choice, not the method's, and are left out
+        n += e * io_bytes * 4 + 2 * bc * io_bytes       # u, delta, z, dout, B, C read
         n += e * 4 * 3 + 2 * bc * 4                     # du, ddelta, dz, dB, dC written
         n += w.dim * w.dstate * 4 + 2 * w.dim * 4       # dA, dD, dbias
     return n
+
+
+# Projections in front of the scan: x_proj (dt_rank + 2 dstate rows) and
+# dt_proj (dim rows), bf16; the step is projections + forward scan.
+PROJ_WORKLOADS = {"mamba130m_layer_proj": ("mamba130m_layer", 48)}
+
+
+def projection_bytes(w, dt_rank):
+    """HBM bytes of the two projections: x read, the weights, dt_low/B/C
+    written, dt_low read again, delta written (bf16)."""
+    M1 = dt_rank + 2 * w.dstate
+    return 2 * (w.batch * w.dim * w.seqlen + M1 * w.dim + w.batch * M1 * w.seqlen
+                + w.dim * dt_rank + w.batch * dt_rank * w.seqlen + w.batch * w.dim * w.seqlen)
 
 
 class ClockSampler:
@@ -245,7 +257,12 @@ def run_ours(args, world, rank, local):
     from selective_state_space_50_b200 import ssm_scan
     from selective_state_space_50_b200.workloads import WORKLOADS, generate, to_torch
 
-    w = WORKLOADS[args.workload]
+    proj = args.workload in PROJ_WORKLOADS
+    if proj:
+        base, dt_rank = PROJ_WORKLOADS[args.workload]
+        w = WORKLOADS[base].replace(name=args.workload)
+    else:
+        w = WORKLOADS[args.workload]
     if args.seqlen:   # shorter sequence of the same workload (profiling small cases)
         w = w.replace(seqlen=args.seqlen, name=f"{w.name}_L{args.seqlen}")
     dev = torch.device("cuda", local)
@@ -255,6 +272,18 @@ def run_ours(args, world, rank, local):
     inp = generate(w_rank, with_dout=fwdbwd)
     dv = to_torch(inp, w_rank, dev)
     shape = ssm_scan.make_shape(w.batch, w.dim, w.seqlen, w.dstate, dv["u"].dtype)
+    if proj:
+        # u is the projections' input x; delta, B and C come from the projections
+        from selective_state_space_50_b200.workloads import generate_projection
+        pinp = generate_projection(w.batch, w.dim, w.seqlen, w.dstate, dt_rank, w_rank.seed)
+        for k in ("x", "W_x", "W_dt"):
+            dv[k] = torch.from_numpy(pinp[k].view(np.int16)).view(torch.bfloat16).to(dev)
+        dv["u"] = dv["x"]
+        bf = dict(device=dev, dtype=torch.bfloat16)
+        dv["delta"] = torch.empty(w.batch, w.dim, w.seqlen, **bf)
+        dv["B"] = torch.empty(w.batch, w.dstate, w.seqlen, **bf)
+        dv["C"] = torch.empty(w.batch, w.dstate, w.seqlen, **bf)
+        dt_low = torch.empty(w.batch, dt_rank, w.seqlen, **bf)
     out = torch.empty_like(dv["u"])
     last = torch.empty(w.batch, w.dim, w.dstate, device=dev, dtype=torch.float32)
     stream = torch.cuda.current_stream(dev)
@@ -279,6 +308,15 @@ def run_ours(args, world, rank, local):
         if bwd_only:   # checkpoints for the timed backward-only steps
             ssm_scan.fwd_raw(shape, dv["u"], dv["delta"], dv["A"], dv["B"], dv["C"], dv["D"],
                              dv["z"], dv["delta_bias"], True, out, last, ck, stream)
+    elif proj:
+        def run_proj():
+            ssm_scan.projections_raw(shape, dt_rank, dv["x"], dv["W_x"], dv["W_dt"], dt_low,
+                                     dv["delta"], dv["B"], dv["C"], stream)
+
+        def fwd():
+            run_proj()
+            ssm_scan.fwd_raw(shape, dv["u"], dv["delta"], dv["A"], dv["B"], dv["C"], dv["D"],
+                             dv["z"], dv["delta_bias"], True, out, last, None, stream)
     else:
         def fwd():
             ssm_scan.fwd_raw(shape, dv["u"], dv["delta"], dv["A"], dv["B"], dv["C"], dv["D"],
@@ -305,11 +343,23 @@ def run_ours(args, world, rank, local):
     t_dev = sum(ms) / 1e3
     t_max = max_over_ranks(t_dev, world)
     elems_all = world * args.steps * w.batch * w.dim * w.seqlen * w.dstate
+    t_proj = None
+    if proj:   # the two projection launches alone, same L2 flush between steps
+        p_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        p_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        for i in range(args.steps):
+            flush.zero_()
+            p_s[i].record(stream)
+            run_proj()
+            p_e[i].record(stream)
+        torch.cuda.synchronize()
+        t_proj = sum(a.elapsed_time(b) for a, b in zip(p_s, p_e)) / 1e3 / args.steps
 
     # ---- end to end through the binding, host buffers, copies inside the step
     e2e_steps = max(5, min(args.steps, 50))
-    host = {k: dv[k].cpu().pin_memory() for k in ("u", "delta", "z", "B", "C", "A", "D",
-                                                   "delta_bias") + (("dout",) if fwdbwd else ())}
+    step_inputs = (("x", "W_x", "W_dt", "z", "A", "D", "delta_bias") if proj else
+                   ("u", "delta", "z", "B", "C", "A", "D", "delta_bias") + (("dout",) if fwdbwd else ()))
+    host = {k: dv[k].cpu().pin_memory() for k in step_inputs}
     out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     du_h = torch.empty(out.shape, dtype=torch.float32).pin_memory() if fwdbwd else None
     h2d = sum(t.numel() * t.element_size() for t in host.values())
@@ -321,6 +371,13 @@ def run_ours(args, world, rank, local):
     def e2e_step():
         for k, t in host.items():
             dtmp[k].copy_(t, non_blocking=True)
+        if proj:
+            d_, B_, C_, _ = ssm_scan.selection_projections(dtmp["x"], dtmp["W_x"], dtmp["W_dt"], w.dstate)
+            o, _, _ = ssm_scan.selective_scan_fwd(dtmp["x"], d_, dtmp["A"], B_, C_, dtmp["D"], dtmp["z"],
+                                                  dtmp["delta_bias"], True, return_last_state=True,
+                                                  out=out)
+            out_h.copy_(o, non_blocking=True)
+            return
         o, _, ckp = ssm_scan.selective_scan_fwd(dtmp["u"], dtmp["delta"], dtmp["A"], dtmp["B"],
                                                 dtmp["C"], dtmp["D"], dtmp["z"], dtmp["delta_bias"],
                                                 True, return_last_state=True, out=out,
@@ -357,7 +414,7 @@ def run_ours(args, world, rank, local):
     alg_bytes = algorithmic_bytes(w, 2 if w.io_dtype == "bf16" else 4, backward=fwdbwd)
     traffic = None
     tp = os.path.join(ROOT, "profiles", "dram_traffic.txt")
-    if os.path.exists(tp) and not fwdbwd:
+    if os.path.exists(tp) and not fwdbwd and not proj:
         with open(tp) as f:
             for line in f:
                 parts = line.split()
@@ -383,10 +440,31 @@ def run_ours(args, world, rank, local):
         "clocks": clk.summary(),
         "e2e": {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": args.steps * (2 if fwdbwd else 1),
+        "gpu_launches": args.steps * (3 if proj else 2 if fwdbwd else 1),
     }
+    if proj:
+        pb = projection_bytes(w, dt_rank)
+        flops = 2 * w.batch * w.seqlen * w.dim * (2 * dt_rank + 2 * w.dstate)
+        line["config"]["dt_rank"] = dt_rank
+        line["config"]["step"] = "x_proj + dt_proj (tcgen05) + forward scan"
+        line["projections"] = {"ms": t_proj * 1e3, "alg_bytes": pb, "flops": flops,
+                               "hbm": {"achieved_gbs": pb / t_proj / 1e9,
+                                       "peak_gbs": float(peaks["hbm_gbs"]),
+                                       "frac": pb / t_proj / 1e9 / float(peaks["hbm_gbs"])},
+                               "tflops": flops / t_proj / 1e12}
     if world == 1 and not args.no_cpu_baseline:
         rate, cores, desc = cpu_oracle_rate(w, inp, args.cpu_budget)
+        if proj:
+            # the oracle's projections on one batch row x 256 steps (all channels)
+            import oracle
+            sl = slice(0, min(256, w.seqlen))
+            t0 = time.perf_counter()
+            oracle.projections(pinp["x_f64"][:1, :, sl], pinp["W_x_f64"], pinp["W_dt_f64"],
+                               dt_rank, w.dstate)
+            tp_s = time.perf_counter() - t0
+            r_proj = w.dim * (sl.stop - sl.start) * w.dstate / tp_s
+            rate = 1.0 / (1.0 / rate + 1.0 / r_proj)
+            desc += f"; projections: 1 batch row x {sl.stop} steps, fp64, {tp_s:.2f} s"
         line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
                                 "sample": desc}
     print(json.dumps(line), flush=True)

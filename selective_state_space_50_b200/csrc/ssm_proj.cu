@@ -19,15 +19,16 @@
 // accumulated in tensor memory, bf16 out.
 //
 // Kernel: one 128 x 128 output tile per CTA, 4 warps.  Lane 0 of warp 0
-// streams 64-deep K slices of A and Bm into a 4-stage shared-memory ring with
-// TMA (128-byte swizzle); lane 0 of warp 1 issues tcgen05.mma (M 128, N 128,
-// K 16) on shared-memory descriptors and frees each stage with
-// tcgen05.commit; warp 2 owns the tensor-memory allocation.  After the last
-// commit all four warps read the accumulator (warp w reads lanes
-// 32w..32w+31, i.e. output rows), convert to bf16 and store 16-byte vectors
-// straight into the output segment that holds each row.  Tiles past M, K or L
-// read zeros (TMA out-of-range fill) and are not stored.  Every wait is
-// bounded; a wait that gives up sets the device error word.
+// streams 64-deep K slices of A and Bm into a shared-memory ring with TMA
+// (128-byte swizzle; 6 stages for x_proj, 1 for dt_proj whose K fits one
+// slice); lane 0 of warp 1 issues tcgen05.mma (M 128, N 128, K 16) on
+// shared-memory descriptors and frees each stage with tcgen05.commit; warp 2
+// owns the tensor-memory allocation.  After the last commit all four warps
+// read the accumulator (warp w reads lanes 32w..32w+31, i.e. output rows),
+// convert to bf16, turn rows into 128-byte row pieces through shared memory
+// and store them into the output segment that holds each row.  Tiles past M,
+// K or L read zeros (TMA out-of-range fill) and are not stored.  Every wait
+// is bounded; a wait that gives up sets the device error word.
 
 #include <cuda_bf16.h>
 
@@ -39,17 +40,32 @@ namespace ssm {
 namespace {
 
 constexpr int kBM = 128, kBN = 128, kBK = 64;        // output tile, K slice
-constexpr int kStages = 4;
 constexpr int kATile = kBM * kBK * 2;                 // [128 rows][64 k] bf16
 constexpr int kBChunk = kBK * 64 * 2;                 // [64 k][64 columns] bf16
 constexpr int kBTile = (kBN / 64) * kBChunk;
 constexpr int kStage = kATile + kBTile;
-constexpr int kBars = kStages * kStage;               // barriers after the ring
-constexpr int kSmem = kBars + (2 * kStages + 1) * 8 + 16;
-constexpr int kSmemAlloc = kSmem + 1024;              // for the 1024-byte alignment
 constexpr int kThreads = 128;
+// Epilogue staging (reuses the ring): per warp 32 rows x 64 columns of bf16,
+// rows padded to 72 elements so that row-wise 16-byte writes spread over the
+// banks.
+constexpr int kStgRow = 72;
+constexpr int kStgWarp = 32 * kStgRow * 2;
 static_assert(kATile % 1024 == 0 && kBChunk % 1024 == 0, "swizzle atoms stay aligned");
 static_assert(kBN % 16 == 0 && kBN >= 16 && kBN <= 256, "UMMA N for M = 128");
+static_assert(4 * kStgWarp <= kStage, "epilogue staging fits in one stage");
+
+// Shared memory of a STAGES-deep ring: the ring, then the barriers and the
+// tensor-memory address.  A one-stage kernel asks for at least 56 KB so that
+// at most four CTAs share an SM: four 128-column accumulators fill its 512
+// tensor-memory columns, and no allocation has to wait.
+template <int STAGES>
+struct ProjSmem {
+    static constexpr int kBars = STAGES * kStage;
+    static constexpr int kUsed = kBars + (2 * STAGES + 1) * 8 + 16 + 1024;
+    static constexpr int kAlloc = kUsed > 56 * 1024 ? kUsed : 56 * 1024;
+    static_assert(kAlloc <= 227 * 1024, "shared memory budget");
+    static_assert(STAGES > 1 || 5 * kAlloc > 228 * 1024, "at most 4 one-stage CTAs per SM");
+};
 
 struct ProjSeg {
     void *ptr;      // [batch][rows][L] bf16
@@ -131,12 +147,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(uint32_t lo, uint32_t hi) {
     return *reinterpret_cast<const uint32_t *>(&v);
 }
 
+template <int kStages>
 __global__ void __launch_bounds__(kThreads, 1)
 proj_gemm_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mB,
                  const ProjParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kBars);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + ProjSmem<kStages>::kBars);
     uint64_t *empty = full + kStages;
     uint64_t *accum = empty + kStages;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accum + 1);
@@ -208,31 +225,46 @@ proj_gemm_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__
     }
 
     // -------------------------------------------------------- epilogue (4 warps)
+    // Warp w holds output rows m0 + 32w .. m0 + 32w + 31 (tensor-memory lanes).
+    // Per 64 columns: each lane converts its row to bf16 into the warp's
+    // staging rows, then the warp writes 4 rows x 128 bytes per instruction.
     const bool ok = __all_sync(0xffffffffu, mbar_wait(accum, 0, p.err));
     tc_fence_after();
     if (ok) {
-        const int m = m0 + warp * 32 + lane;
-        __nv_bfloat16 *row = nullptr;         // this thread's output row, if it has one
-#pragma unroll
-        for (int i = 0; i < 3; ++i) {
-            const int r0 = p.seg[i].row0, nr = p.seg[i].rows;
-            if (i < p.nseg && m < p.M && m >= r0 && m < r0 + nr)
-                row = static_cast<__nv_bfloat16 *>(p.seg[i].ptr) + ((size_t)b * nr + (m - r0)) * (size_t)p.L;
-        }
+        __nv_bfloat16 *stg = reinterpret_cast<__nv_bfloat16 *>(smem + warp * kStgWarp);
+        const int srow = lane / 8, schunk = lane % 8;     // write-out: row within 4, 16-byte chunk
 #pragma unroll 1
-        for (int c = 0; c < kBN / 16; ++c) {
-            uint32_t r[16];
-            tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(c * 16), r);
-            const int n = n0 + c * 16;
-            if (row) {
+        for (int h = 0; h < kBN / 64; ++h) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t r[16];
+                tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(h * 64 + c * 16), r);
                 uint4 v0, v1;
                 v0.x = pack_bf16x2(r[0], r[1]);   v0.y = pack_bf16x2(r[2], r[3]);
                 v0.z = pack_bf16x2(r[4], r[5]);   v0.w = pack_bf16x2(r[6], r[7]);
                 v1.x = pack_bf16x2(r[8], r[9]);   v1.y = pack_bf16x2(r[10], r[11]);
                 v1.z = pack_bf16x2(r[12], r[13]); v1.w = pack_bf16x2(r[14], r[15]);
-                if (n + 8 <= p.L) *reinterpret_cast<uint4 *>(row + n) = v0;
-                if (n + 16 <= p.L) *reinterpret_cast<uint4 *>(row + n + 8) = v1;
+                *reinterpret_cast<uint4 *>(stg + lane * kStgRow + c * 16) = v0;
+                *reinterpret_cast<uint4 *>(stg + lane * kStgRow + c * 16 + 8) = v1;
             }
+            __syncwarp();
+            const int n = n0 + h * 64 + schunk * 8;
+#pragma unroll
+            for (int it = 0; it < 8; ++it) {
+                const int rl = it * 4 + srow;                 // row within the warp's 32
+                const int m = m0 + warp * 32 + rl;
+                __nv_bfloat16 *row = nullptr;
+#pragma unroll
+                for (int i = 0; i < 3; ++i) {
+                    const int r0 = p.seg[i].row0, nr = p.seg[i].rows;
+                    if (i < p.nseg && m < p.M && m >= r0 && m < r0 + nr)
+                        row = static_cast<__nv_bfloat16 *>(p.seg[i].ptr) + ((size_t)b * nr + (m - r0)) * (size_t)p.L;
+                }
+                if (row && n + 8 <= p.L)
+                    *reinterpret_cast<uint4 *>(row + n) =
+                        *reinterpret_cast<const uint4 *>(stg + rl * kStgRow + schunk * 8);
+            }
+            __syncwarp();
         }
     }
     tc_fence_before();
@@ -240,17 +272,28 @@ proj_gemm_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__
     if (warp == 2) tmem_dealloc(tmem, kBN);
 }
 
+template <int STAGES>
 cudaError_t launch_proj_gemm(const CUtensorMap &mA, const CUtensorMap &mB, const ProjParams &p, int batch,
                              cudaStream_t stream) {
+    constexpr int smem = ProjSmem<STAGES>::kAlloc;
     static bool attr_done = false;
     if (!attr_done) {
-        cudaError_t e = cudaFuncSetAttribute(proj_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
+        cudaError_t e = cudaFuncSetAttribute(proj_gemm_kernel<STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         attr_done = true;
     }
     const dim3 grid((unsigned)((p.L + kBN - 1) / kBN), (unsigned)((p.M + kBM - 1) / kBM), (unsigned)batch);
-    proj_gemm_kernel<<<grid, kThreads, kSmemAlloc, stream>>>(mA, mB, p);
+    proj_gemm_kernel<STAGES><<<grid, kThreads, smem, stream>>>(mA, mB, p);
     return cudaGetLastError();
+}
+
+// A deep ring when the contraction is long (x_proj streams the activations
+// through it); a single stage, with up to four CTAs per SM overlapping each
+// other's loads, MMAs and stores, when one K slice covers it (dt_proj).
+cudaError_t launch_proj_any(const CUtensorMap &mA, const CUtensorMap &mB, const ProjParams &p, int batch,
+                            cudaStream_t stream) {
+    return p.K <= kBK ? launch_proj_gemm<1>(mA, mB, p, batch, stream)
+                      : launch_proj_gemm<6>(mA, mB, p, batch, stream);
 }
 
 }  // namespace
@@ -272,7 +315,7 @@ cudaError_t launch_projections(const ProjShape &s, const void *x, const void *W_
     p.seg[2] = {C, R + N, N};
     p.nseg = 3;
     p.M = M1; p.K = s.dim; p.L = s.seqlen; p.err = err;
-    cudaError_t e = launch_proj_gemm(mA, mB, p, s.batch, stream);
+    cudaError_t e = launch_proj_any(mA, mB, p, s.batch, stream);
     if (e != cudaSuccess) return e;
     // dt_proj: A = W_dt [D x R], Bm = dt_low [batch][R][L]
     if (!make_tma_map_2d(&mA, W_dt, true, (uint64_t)s.dim, (uint64_t)R, kBK, kBM, true) ||
@@ -282,7 +325,7 @@ cudaError_t launch_projections(const ProjShape &s, const void *x, const void *W_
     q.seg[0] = {delta, 0, s.dim};
     q.nseg = 1;
     q.M = s.dim; q.K = R; q.L = s.seqlen; q.err = err;
-    return launch_proj_gemm(mA, mB, q, s.batch, stream);
+    return launch_proj_any(mA, mB, q, s.batch, stream);
 }
 
 }  // namespace ssm
