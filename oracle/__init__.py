@@ -181,3 +181,35 @@ def projections(x, W_x, W_dt, dt_rank: int, dstate: int, store_low_bf16: bool = 
     delta = np.matmul(W_dt[None, :, :], low)             # [b, D, L]
     return (np.ascontiguousarray(dt_low), np.ascontiguousarray(delta),
             np.ascontiguousarray(B), np.ascontiguousarray(C))
+
+
+# ------------------------------------------------------------------ sequence segments
+# A sequence split into segments is reassembled from per-segment summaries with
+# the associative operator of the two-level scan (booiljung.github.io, "3.2
+# 선택적 스캔(Selective Scan) 알고리즘", §2.2: (a_j, b_j) • (a_i, b_i) =
+# (a_j a_i, a_j b_i + b_j)).  Segment s, run from a zero state, ends in state
+# e_s; its decay product over the segment is prod_t exp(Δ_t A) = exp(A Σ_t Δ_t).
+
+def delta_sums(delta, delta_bias=None, delta_softplus=True) -> np.ndarray:
+    """Σ_t Δ_t per (batch, channel) of one segment: [b, D, L] -> [b, D]."""
+    r = _f64(delta) + (0.0 if delta_bias is None else _f64(delta_bias)[None, :, None])
+    dt = np.logaddexp(0.0, r) if delta_softplus else r
+    return dt.sum(axis=2)
+
+
+def combine_carries(A, dsums, h_ends, h0=None) -> np.ndarray:
+    """Exclusive scan of segment summaries in sequence order.
+
+    A [D, N]; dsums [S, b, D]; h_ends [S, b, D, N] (each segment's end state
+    from a zero start).  Returns h_in [S, b, D, N], the state entering each
+    segment: h_in[0] = h0 (zero if None), h_in[s+1] = exp(A dsums[s]) h_in[s]
+    + h_ends[s]."""
+    A, dsums, h_ends = map(_f64, (A, dsums, h_ends))
+    S = dsums.shape[0]
+    out = np.empty_like(h_ends)
+    h = np.zeros_like(h_ends[0]) if h0 is None else _f64(h0).copy()
+    for s in range(S):
+        out[s] = h
+        decay = np.exp(dsums[s][:, :, None] * A[None, :, :])
+        h = decay * h + h_ends[s]
+    return out

@@ -442,3 +442,45 @@ def test_adjoint_directional_derivative_larger_case():
     fd = (at(1) - at(-1)) / (2 * eps)
     an = sum(float((g[GRAD_OF[k]] * v[k]).sum()) for k in GRAD_OF)
     assert abs(fd - an) <= 1e-7 * max(1.0, abs(an))
+
+
+@pytest.mark.parametrize("cuts", [(0, 200), (0, 64, 200), (0, 1, 97, 150, 200)])
+def test_segments_reassembled_by_carries_equal_the_whole_scan(cuts):
+    """Split-sequence invariant behind sequence sharding: each segment run from
+    a zero state gives (Σ Δ, end state); combine_carries turns those into the
+    state entering every segment, and re-running each segment from it equals
+    the forward over the whole sequence (out and final state)."""
+    r = rng(12)
+    batch, dim, N, L = 2, 3, 4, 200
+    u = r.standard_normal((batch, dim, L))
+    delta = r.standard_normal((batch, dim, L))
+    A = -np.exp(r.standard_normal((dim, N)))
+    B = r.standard_normal((batch, N, L))
+    C = r.standard_normal((batch, N, L))
+    D = r.uniform(0.5, 1.5, dim)
+    z = r.standard_normal((batch, dim, L))
+    bias = r.uniform(-1, 1, dim)
+    h0 = r.standard_normal((batch, dim, N))
+    want, wlast = oracle.fwd(u, delta, A, B, C, D, z, bias, True, h0=h0)
+    segs = list(zip(cuts[:-1], cuts[1:]))
+    ds, ends = [], []
+    for a, b in segs:
+        _, e = oracle.fwd(u[..., a:b], delta[..., a:b], A, B[..., a:b], C[..., a:b], D,
+                          z[..., a:b], bias, True)
+        ds.append(oracle.delta_sums(delta[..., a:b], bias, True))
+        ends.append(e)
+    hin = oracle.combine_carries(A, np.stack(ds), np.stack(ends), h0)
+    got = np.empty_like(want)
+    for s, (a, b) in enumerate(segs):
+        got[..., a:b], last = oracle.fwd(u[..., a:b], delta[..., a:b], A, B[..., a:b], C[..., a:b],
+                                         D, z[..., a:b], bias, True, h0=hin[s])
+    np.testing.assert_allclose(got, want, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(last, wlast, rtol=1e-11, atol=1e-12)
+
+
+def test_delta_sums_softplus_and_raw():
+    d = np.array([[[0.0, 1.0, -30.0]]])
+    np.testing.assert_allclose(oracle.delta_sums(d, None, False), [[-29.0]])
+    np.testing.assert_allclose(oracle.delta_sums(d, np.array([1.0]), True),
+                               [[np.log1p(np.e) + np.log1p(np.e ** 2) + np.log1p(np.exp(-29.0))]],
+                               rtol=1e-14)
