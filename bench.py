@@ -308,6 +308,52 @@ def run_ours(args, world, rank, local):
         if bwd_only:   # checkpoints for the timed backward-only steps
             ssm_scan.fwd_raw(shape, dv["u"], dv["delta"], dv["A"], dv["B"], dv["C"], dv["D"],
                              dv["z"], dv["delta_bias"], True, out, last, ck, stream)
+    elif args.segments > 1:
+        # the sequence cut into S segments, run with the sharded protocol on
+        # this one GPU (pass 1 over all segments, combine, pass 2 over 1..S-1)
+        from selective_state_space_50_b200 import seqpar
+        S = args.segments
+        if w.seqlen % S:
+            raise SystemExit("--segments must divide seqlen")
+        Ls = w.seqlen // S
+        seg_shape = ssm_scan.make_shape(w.batch, w.dim, Ls, w.dstate, dv["u"].dtype)
+        pieces = [{k: dv[k][..., s_ * Ls:(s_ + 1) * Ls].contiguous() for k in ("u", "delta", "z", "B", "C")}
+                  for s_ in range(S)]
+        f32 = dict(device=dev, dtype=torch.float32)
+        seg_out = [torch.empty_like(pc["u"]) for pc in pieces]
+        seg_last = torch.empty(S, w.batch, w.dim, w.dstate, **f32)
+        seg_dsum = torch.empty(S, w.batch, w.dim, **f32)
+        h_in = torch.empty(S, w.batch, w.dim, w.dstate, **f32)
+        mid = S // 2
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+        seg_times = []
+
+        def run_segment(s_, h0, timed=False):
+            pc = pieces[s_]
+            ssm_scan.fwd_segment_raw(seg_shape, pc["u"], pc["delta"], dv["A"], pc["B"], pc["C"], dv["D"],
+                                     pc["z"], dv["delta_bias"], True, h0, seg_out[s_], seg_last[s_],
+                                     None, seg_dsum[s_] if h0 is None else None, stream)
+            return seg_out[s_], seg_last[s_], seg_dsum[s_]
+
+        def fwd(record=False):
+            for s_ in range(S):
+                if record and s_ == mid:
+                    ev[0].record(stream)
+                run_segment(s_, None)
+                if record and s_ == mid:
+                    ev[1].record(stream)
+            if record:
+                ev[2].record(stream)
+            ssm_scan.combine_carries_raw(S, w.batch, w.dim, w.dstate, dv["A"], seg_dsum, seg_last, None,
+                                         h_in, stream)
+            if record:
+                ev[3].record(stream)
+            for s_ in range(1, S):
+                if record and s_ == mid:
+                    ev[4].record(stream)
+                run_segment(s_, h_in[s_])
+                if record and s_ == mid:
+                    ev[5].record(stream)
     elif proj:
         def run_proj():
             ssm_scan.projections_raw(shape, dt_rank, dv["x"], dv["W_x"], dv["W_dt"], dt_low,
@@ -343,6 +389,21 @@ def run_ours(args, world, rank, local):
     t_dev = sum(ms) / 1e3
     t_max = max_over_ranks(t_dev, world)
     elems_all = world * args.steps * w.batch * w.dim * w.seqlen * w.dstate
+    seg_info = None
+    if args.segments > 1:   # one segment's critical path: its pass 1, the combine, its pass 2
+        parts = []
+        for _ in range(max(3, min(args.steps, 20))):
+            flush.zero_()
+            fwd(record=True)
+            torch.cuda.synchronize()
+            parts.append((ev[0].elapsed_time(ev[1]), ev[2].elapsed_time(ev[3]), ev[4].elapsed_time(ev[5])))
+        p1, cb, p2 = (statistics.median(x[i] for x in parts) for i in range(3))
+        seg_info = {"n": args.segments, "seqlen_per_segment": w.seqlen // args.segments,
+                    "pass1_ms": p1, "combine_ms": cb, "pass2_ms": p2, "per_rank_ms": p1 + cb + p2,
+                    "exchange_bytes_per_rank": w.batch * w.dim * (w.dstate + 1) * 4,
+                    "note": "segments run in turn on one GPU; per_rank_ms is one segment's critical "
+                            "path (pass 1 + combine + pass 2, each timed with CUDA events on this GPU); "
+                            "the all-gather of the summaries between ranks is not included"}
     t_proj = None
     if proj:   # the two projection launches alone, same L2 flush between steps
         p_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
@@ -371,6 +432,12 @@ def run_ours(args, world, rank, local):
     def e2e_step():
         for k, t in host.items():
             dtmp[k].copy_(t, non_blocking=True)
+        if args.segments > 1:
+            o, _ = seqpar.cuda_forward_segments(dtmp["u"], dtmp["delta"], dtmp["A"], dtmp["B"], dtmp["C"],
+                                                dtmp["D"], dtmp["z"], dtmp["delta_bias"], True,
+                                                nseg=args.segments)
+            out_h.copy_(o, non_blocking=True)
+            return
         if proj:
             d_, B_, C_, _ = ssm_scan.selection_projections(dtmp["x"], dtmp["W_x"], dtmp["W_dt"], w.dstate)
             o, _, _ = ssm_scan.selective_scan_fwd(dtmp["x"], d_, dtmp["A"], B_, C_, dtmp["D"], dtmp["z"],
@@ -440,8 +507,13 @@ def run_ours(args, world, rank, local):
         "clocks": clk.summary(),
         "e2e": {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": args.steps * (3 if proj else 2 if fwdbwd else 1),
+        "gpu_launches": args.steps * (3 if proj else 2 if fwdbwd else
+                                      (3 * args.segments if args.segments > 1 else 1)),
     }
+    if seg_info:
+        line["segments"] = seg_info
+        line["config"]["step"] = (f"sequence cut into {args.segments} segments: pass 1 over all, "
+                                  f"carry combine, pass 2 over segments 1..{args.segments - 1}")
     if proj:
         pb = projection_bytes(w, dt_rank)
         flops = 2 * w.batch * w.seqlen * w.dim * (2 * dt_rank + 2 * w.dstate)
@@ -597,6 +669,8 @@ def main():
                     help="workload to time (default: the Mamba-130M layer shape)")
     ap.add_argument("--seqlen", type=int, default=0,
                     help="override the workload's sequence length (for profiling small cases)")
+    ap.add_argument("--segments", type=int, default=1,
+                    help="run the forward as S sequence segments with the sharded protocol")
     ap.add_argument("--decode", action="store_true",
                     help="time the single-step recurrent update instead of the scan")
     args = ap.parse_args()

@@ -294,6 +294,55 @@ ssm_status_t ssm_device_error_status(void *stream);
 ssm_status_t ssm_selftest_wait_timeout(void *stream);
 
 /*
+ * Forward over one SEGMENT of a longer sequence (sequence sharding).
+ *
+ * The same forward as ssm_selective_scan_fwd_ex, over seqlen steps of a
+ * segment, started from the state h0 ([batch][dim][dstate] float32, the state
+ * after the previous segment's last step; NULL means zeros, as at the start of
+ * a sequence).  last_state receives the state after the segment's last step.
+ * delta_sum (nullable, [batch][dim] float32) receives Σ_t Δ_t over the
+ * segment, with Δ exactly as the scan forms it (softplus of delta + bias when
+ * enabled).
+ *
+ * A sequence cut into segments 0..S-1 is reassembled with the associative
+ * operator of the two-level scan (booiljung.github.io, "3.2 선택적 스캔
+ * (Selective Scan) 알고리즘과 정보의 압축 및 선별", §2.2):
+ *   1. run every segment from h0 = NULL, keeping last_state (e_s) and
+ *      delta_sum (Σ_s);
+ *   2. ssm_scan_combine_carries turns (Σ_s, e_s) into the state entering each
+ *      segment;
+ *   3. run segments 1..S-1 again from those states; their out and last_state
+ *      then equal the forward over the whole sequence.
+ * Segment 0's first run is already final.  The checkpoints written from
+ * h0 != NULL are the states of that run; the backward entry points assume a
+ * zero initial state and must not be given them.
+ * Errors: as ssm_selective_scan_fwd_ex; h0 may not alias last_state or ckpt.
+ */
+ssm_status_t ssm_selective_scan_fwd_segment(const ssm_shape_t *shape, const ssm_options_t *opts,
+                                            const void *u, const void *delta, const float *A,
+                                            const void *B, const void *C, const float *D,
+                                            const void *z, const float *delta_bias, const float *h0,
+                                            void *out, float *last_state, float *ckpt,
+                                            float *delta_sum, void *stream);
+
+/*
+ * Exclusive scan of segment summaries, in sequence order, for S = nseg
+ * segments of one sequence batch ([batch][dim] channel rows, dstate states):
+ *   h_in[0] = h0 (zeros if NULL)
+ *   h_in[s+1][r][n] = exp(A[r % dim][n] · delta_sums[s][r]) · h_in[s][r][n]
+ *                     + h_ends[s][r][n]
+ * exp(A Σ_t Δ_t) is the product of the segment's per-step factors exp(Δ_t A).
+ * Layouts (float32, device): A [dim][dstate], delta_sums [nseg][batch][dim],
+ * h_ends and h_in [nseg][batch][dim][dstate], h0 [batch][dim][dstate].
+ * One thread per (row, state); asynchronous on `stream`.
+ * Errors: SSM_ERR_INVALID_ARG (sizes < 1, NULL/host/misaligned pointers,
+ * h_in aliasing an input), SSM_ERR_CUDA.
+ */
+ssm_status_t ssm_scan_combine_carries(int nseg, int batch, int dim, int dstate, const float *A,
+                                      const float *delta_sums, const float *h_ends,
+                                      const float *h0, float *h_in, void *stream);
+
+/*
  * Selection projections: the per-token Linear layers that make the scan's
  * step size, B and C functions of its input x (= u of the scan).
  * booiljung.github.io, "3.2 선택적 스캔(Selective Scan) 알고리즘과 정보의 압축

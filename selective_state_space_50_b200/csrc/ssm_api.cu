@@ -158,11 +158,15 @@ ssm_status_t ssm_selective_scan_bwd_scratch_bytes(const ssm_shape_t *shape, int 
     return ok();
 }
 
-ssm_status_t ssm_selective_scan_fwd_ex(const ssm_shape_t *shape, const ssm_options_t *opts,
-                                       const void *u, const void *delta, const float *A,
-                                       const void *B, const void *C, const float *D, const void *z,
-                                       const float *delta_bias, void *out, float *last_state,
-                                       float *ckpt, void *stream) {
+}  // extern "C"
+
+namespace {
+
+// The forward behind ssm_selective_scan_fwd_ex and ssm_selective_scan_fwd_segment.
+ssm_status_t fwd_impl(const ssm_shape_t *shape, const ssm_options_t *opts, const void *u,
+                      const void *delta, const float *A, const void *B, const void *C,
+                      const float *D, const void *z, const float *delta_bias, const float *h0,
+                      void *out, float *last_state, float *ckpt, float *delta_sum, void *stream) {
     SSM_TRY(check_shape(shape));
     SSM_TRY(check_options(opts));
     const size_t es = esize(shape->io_dtype);
@@ -174,15 +178,19 @@ ssm_status_t ssm_selective_scan_fwd_ex(const ssm_shape_t *shape, const ssm_optio
     SSM_TRY(check_ptr(D, "D", 4, false));
     SSM_TRY(check_ptr(z, "z", es, false));
     SSM_TRY(check_ptr(delta_bias, "delta_bias", 4, false));
+    SSM_TRY(check_ptr(h0, "h0", 4, false));
     SSM_TRY(check_ptr(out, "out", es, true));
     SSM_TRY(check_ptr(last_state, "last_state", 4, false));
     SSM_TRY(check_ptr(ckpt, "ckpt", 4, false));
+    SSM_TRY(check_ptr(delta_sum, "delta_sum", 4, false));
     if (out == u || out == delta || out == z || out == B || out == C)
         return fail(SSM_ERR_INVALID_ARG, "out may not alias an input");
+    if (h0 && (h0 == last_state || (const void *)h0 == (const void *)ckpt))
+        return fail(SSM_ERR_INVALID_ARG, "h0 may not alias last_state or ckpt");
 
     ssm::FwdParams p{};
     p.u = u; p.delta = delta; p.A = A; p.B = B; p.C = C; p.D = D; p.z = z;
-    p.delta_bias = delta_bias; p.out = out; p.last_state = last_state; p.ckpt = ckpt;
+    p.delta_bias = delta_bias; p.out = out; p.last_state = last_state; p.ckpt = ckpt; p.h0 = h0;
     p.batch = shape->batch; p.dim = shape->dim; p.L = shape->seqlen; p.N = shape->dstate;
     p.n_ckpt = n_ckpt(shape);
     p.softplus = opts->delta_softplus != 0;
@@ -192,6 +200,55 @@ ssm_status_t ssm_selective_scan_fwd_ex(const ssm_shape_t *shape, const ssm_optio
                aligned16(B) && aligned16(C) && aligned16(out) && (!z || aligned16(z));
     cudaError_t e = ssm::launch_fwd(p, false, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "ssm_selective_scan_fwd launch");
+    if (delta_sum) {
+        e = ssm::launch_delta_sum(p, delta_sum, static_cast<cudaStream_t>(stream));
+        if (e != cudaSuccess) return cuda_fail(e, "ssm_selective_scan_fwd_segment delta sums");
+    }
+    return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+ssm_status_t ssm_selective_scan_fwd_ex(const ssm_shape_t *shape, const ssm_options_t *opts,
+                                       const void *u, const void *delta, const float *A,
+                                       const void *B, const void *C, const float *D, const void *z,
+                                       const float *delta_bias, void *out, float *last_state,
+                                       float *ckpt, void *stream) {
+    return fwd_impl(shape, opts, u, delta, A, B, C, D, z, delta_bias, nullptr, out, last_state, ckpt,
+                    nullptr, stream);
+}
+
+ssm_status_t ssm_selective_scan_fwd_segment(const ssm_shape_t *shape, const ssm_options_t *opts,
+                                            const void *u, const void *delta, const float *A,
+                                            const void *B, const void *C, const float *D,
+                                            const void *z, const float *delta_bias, const float *h0,
+                                            void *out, float *last_state, float *ckpt,
+                                            float *delta_sum, void *stream) {
+    return fwd_impl(shape, opts, u, delta, A, B, C, D, z, delta_bias, h0, out, last_state, ckpt,
+                    delta_sum, stream);
+}
+
+ssm_status_t ssm_scan_combine_carries(int nseg, int batch, int dim, int dstate, const float *A,
+                                      const float *delta_sums, const float *h_ends, const float *h0,
+                                      float *h_in, void *stream) {
+    if (nseg < 1 || batch < 1 || dim < 1 || dstate < 1)
+        return fail(SSM_ERR_INVALID_ARG, "nseg, batch, dim, dstate must be >= 1");
+    const long long P = (long long)batch * dim;
+    if ((long long)nseg * P * dstate >= (1LL << 40))
+        return fail(SSM_ERR_UNSUPPORTED, "nseg*batch*dim*dstate too large");
+    SSM_TRY(check_ptr(A, "A", 4, true));
+    SSM_TRY(check_ptr(delta_sums, "delta_sums", 4, true));
+    SSM_TRY(check_ptr(h_ends, "h_ends", 4, true));
+    SSM_TRY(check_ptr(h0, "h0", 4, false));
+    SSM_TRY(check_ptr(h_in, "h_in", 4, true));
+    if ((const void *)h_in == (const void *)h_ends || (const void *)h_in == (const void *)delta_sums ||
+        (h0 && h_in == h0))
+        return fail(SSM_ERR_INVALID_ARG, "h_in may not alias an input");
+    cudaError_t e = ssm::launch_combine_carries(nseg, P, dim, dstate, A, delta_sums, h_ends, h0, h_in,
+                                                static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "ssm_scan_combine_carries launch");
     return ok();
 }
 

@@ -102,7 +102,7 @@ fwd_kernel(const FwdParams p) {
 #pragma unroll
     for (int s = 0; s < NS; ++s) {
         A2[s] = live ? p.A[(size_t)d * N + g * NS + s] * SSM_LOG2E : 0.f;
-        h[s] = 0.f;
+        h[s] = (live && p.h0) ? p.h0[((size_t)b * p.dim + d) * N + g * NS + s] : 0.f;
     }
 
     const size_t row_bd0 = (size_t)b * p.dim;

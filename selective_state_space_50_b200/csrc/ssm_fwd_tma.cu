@@ -60,6 +60,7 @@ constexpr int align128(int x) { return (x + 127) / 128 * 128; }
 
 struct TmaFwdParams {
     const float *A, *D, *delta_bias;
+    const float *h0;    // [P][N] state before step 0; NULL: zeros
     void *out;
     float *last_state, *ckpt;
     int P;          // batch * dim channel rows
@@ -275,7 +276,7 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
             for (int j = 0; j < NS; ++j) {
                 const float a = live ? p.A[(size_t)d * N + g * NS + j] * SSM_LOG2E : 0.f;
                 A2d[j] = make_float2(a, a);
-                h[j] = 0.f;
+                h[j] = (live && p.h0) ? p.h0[(size_t)row * N + g * NS + j] : 0.f;
                 neg = neg && a <= 0.f;
             }
             poly_ok = __all_sync(0xffffffffu, neg);
@@ -484,7 +485,7 @@ cudaError_t launch_cfg(const FwdParams &fp, cudaStream_t stream) {
         return cudaErrorInvalidValue;
     TmaFwdParams p{};
     p.A = fp.A; p.D = fp.D; p.delta_bias = fp.delta_bias; p.out = fp.out;
-    p.last_state = fp.last_state; p.ckpt = fp.ckpt;
+    p.last_state = fp.last_state; p.ckpt = fp.ckpt; p.h0 = fp.h0;
     p.P = P; p.dim = fp.dim; p.L = fp.L; p.n_ckpt = fp.n_ckpt;
     p.softplus = fp.softplus; p.has_z = fp.z != nullptr; p.rows_max = rows_max;
     p.err = device_error_word();

@@ -18,6 +18,7 @@ struct FwdParams {
     const float *delta_bias;
     void *out;
     float *last_state, *ckpt;
+    const float *h0;  // [batch][dim][N] state before step 0; NULL: zeros
     int batch, dim, L, N, n_ckpt;
     int softplus;
     int zoh;      // zero-order-hold B̄ (general kernels only)
@@ -66,6 +67,14 @@ struct ProjShape {
 };
 cudaError_t launch_projections(const ProjShape &s, const void *x, const void *W_x, const void *W_dt,
                                void *dt_low, void *delta, void *B, void *C, cudaStream_t stream);
+
+// Sequence segments (ssm_seg.cu).  delta_sum[b][d] = Σ_t Δ_t over the
+// segment; combine_carries turns per-segment (Σ Δ, end state) pairs into the
+// state entering each segment.
+cudaError_t launch_delta_sum(const FwdParams &p, float *delta_sum, cudaStream_t stream);
+cudaError_t launch_combine_carries(int nseg, long long P, int dim, int N, const float *A,
+                                   const float *dsums, const float *h_ends, const float *h0,
+                                   float *h_in, cudaStream_t stream);
 
 // Single-step recurrent update (ssm_step.cu).
 cudaError_t launch_state_update(const StepParams &p, cudaStream_t stream);

@@ -28,7 +28,8 @@ EXPORTS = ("ssm_version", "ssm_last_error_string", "ssm_selective_scan_ckpt_byte
            "ssm_selective_scan_bwd_noalloc", "ssm_selective_state_update",
            "ssm_selective_scan_fwd_ex", "ssm_selective_scan_bwd_ex",
            "ssm_selective_state_update_ex", "ssm_selftest_wait_timeout",
-           "ssm_selection_projections")
+           "ssm_selection_projections", "ssm_selective_scan_fwd_segment",
+           "ssm_scan_combine_carries")
 SSM_DISC_DELTA_B, SSM_DISC_ZOH = 0, 1
 NOALLOC_SCRATCH_BYTES = 32 << 20  # SSM_NOALLOC_SCRATCH_BYTES in include/ssm_scan.h
 
@@ -93,6 +94,10 @@ def load_library(path: str = LIB_PATH):
     lib.ssm_selftest_wait_timeout.restype = i
     lib.ssm_selection_projections.argtypes = [sp, i] + [vp] * 8
     lib.ssm_selection_projections.restype = i
+    lib.ssm_selective_scan_fwd_segment.argtypes = [sp, op] + [vp] * 14
+    lib.ssm_selective_scan_fwd_segment.restype = i
+    lib.ssm_scan_combine_carries.argtypes = [i, i, i, i] + [vp] * 5 + [vp]
+    lib.ssm_scan_combine_carries.restype = i
     _lib = lib
     return lib
 
@@ -316,3 +321,54 @@ def selection_projections(x, W_x, W_dt, dstate: int, stream=None):
     C = torch.empty(batch, dstate, L, **kw)
     projections_raw(shape, dt_rank, x, W_x, W_dt, dt_low, delta, B, C, stream)
     return delta, B, C, dt_low
+
+
+def fwd_segment_raw(shape: Shape, u, delta, A, B, C, D, z, delta_bias, delta_softplus: bool, h0,
+                    out, last_state, ckpt=None, delta_sum=None, stream=None, zoh: bool = False):
+    """Direct call of ssm_selective_scan_fwd_segment."""
+    o = _opts(delta_softplus, zoh)
+    _check(load_library().ssm_selective_scan_fwd_segment(
+        ctypes.byref(shape), ctypes.byref(o), _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C),
+        _ptr(D), _ptr(z), _ptr(delta_bias), _ptr(h0), _ptr(out), _ptr(last_state), _ptr(ckpt),
+        _ptr(delta_sum), _stream_ptr(stream)))
+
+
+def combine_carries_raw(nseg, batch, dim, dstate, A, delta_sums, h_ends, h0, h_in, stream=None):
+    """Direct call of ssm_scan_combine_carries."""
+    _check(load_library().ssm_scan_combine_carries(
+        int(nseg), int(batch), int(dim), int(dstate), _ptr(A), _ptr(delta_sums), _ptr(h_ends),
+        _ptr(h0), _ptr(h_in), _stream_ptr(stream)))
+
+
+def selective_scan_fwd_segment(u, delta, A, B, C, D=None, z=None, delta_bias=None,
+                               delta_softplus: bool = True, h0=None, out=None, stream=None,
+                               zoh: bool = False):
+    """Forward over one segment of a sequence from state h0 ([batch, dim,
+    dstate] float32, None = zeros).  Returns (out, last_state, delta_sum)
+    with delta_sum [batch, dim] = Σ_t Δ_t over the segment."""
+    io = u.dtype
+    for t, n in ((u, "u"), (delta, "delta"), (B, "B"), (C, "C"), (z, "z")):
+        _need(t, n, io)
+    for t, n in ((A, "A"), (D, "D"), (delta_bias, "delta_bias"), (h0, "h0")):
+        _need(t, n, torch.float32)
+    shape = _shape_of(u, A)
+    if out is None:
+        out = torch.empty_like(u)
+    f32 = dict(device=u.device, dtype=torch.float32)
+    last = torch.empty(shape.batch, shape.dim, shape.dstate, **f32)
+    dsum = torch.empty(shape.batch, shape.dim, **f32)
+    fwd_segment_raw(shape, u, delta, A, B, C, D, z, delta_bias, delta_softplus, h0, out, last,
+                    None, dsum, stream, zoh)
+    return out, last, dsum
+
+
+def combine_carries(A, delta_sums, h_ends, h0=None, stream=None):
+    """States entering each of S segments from their summaries: delta_sums
+    [S, batch, dim], h_ends [S, batch, dim, dstate] (float32, device).
+    Returns h_in [S, batch, dim, dstate]."""
+    for t, n in ((A, "A"), (delta_sums, "delta_sums"), (h_ends, "h_ends"), (h0, "h0")):
+        _need(t, n, torch.float32)
+    S, batch, dim, dstate = h_ends.shape
+    h_in = torch.empty_like(h_ends)
+    combine_carries_raw(S, batch, dim, dstate, A, delta_sums, h_ends, h0, h_in, stream)
+    return h_in

@@ -78,3 +78,68 @@ def test_reference_arm_under_torchrun():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def _seqpar_worker(rank, world, port, out_q):
+    """One rank of the sequence-sharded forward protocol over gloo, with the
+    oracle doing each segment's scan (this test checks the exchange: which
+    rank runs what, gather order, carry-in selection)."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import oracle
+    from selective_state_space_50_b200 import seqpar
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        r = np.random.default_rng(5)
+        batch, dim, N, L = 2, 3, 4, 60
+        u, delta, z = r.standard_normal((3, batch, dim, L))
+        A = -np.exp(r.standard_normal((dim, N)))
+        B, C = r.standard_normal((2, batch, N, L))
+        D = r.uniform(0.5, 1.5, dim)
+        bias = r.uniform(-1, 1, dim)
+        Ls = L // world
+        sl = slice(rank * Ls, (rank + 1) * Ls)
+        calls = []
+
+        def run_segment(h0):
+            calls.append(h0 is not None)
+            out, last = oracle.fwd(u[..., sl], delta[..., sl], A, B[..., sl], C[..., sl], D,
+                                   z[..., sl], bias, True, h0=None if h0 is None else h0.numpy())
+            return out, torch.from_numpy(last), torch.from_numpy(oracle.delta_sums(delta[..., sl], bias))
+
+        def gather(x):
+            parts = [torch.empty_like(x) for _ in range(world)]
+            dist.all_gather(parts, x)
+            return torch.stack(parts)
+
+        def combine(ds, es):
+            return torch.from_numpy(oracle.combine_carries(A, ds.numpy(), es.numpy()))
+
+        out, last = seqpar.forward_rank(rank, run_segment, gather, combine)
+        want, wlast = oracle.fwd(u, delta, A, B, C, D, z, bias, True)
+        ok_out = np.allclose(out, want[..., sl], rtol=1e-11, atol=1e-12)
+        ok_last = rank != world - 1 or np.allclose(last.numpy(), wlast, rtol=1e-11, atol=1e-12)
+        out_q.put((rank, bool(ok_out), bool(ok_last), calls))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_sequence_sharded_forward_protocol_gloo(world):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_seqpar_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=180)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(world))
+    for rank, ok_out, ok_last, calls in res:
+        assert ok_out and ok_last, rank
+        # pass 1 from zeros everywhere; pass 2 from the carry-in on ranks > 0 only
+        assert calls == ([False] if rank == 0 else [False, True])
