@@ -81,11 +81,9 @@ struct BwdLayout {
     static constexpr int W = 8;                                        // window = checkpoint chunk
     static constexpr int NWIN = TT / W;
     static constexpr int WS = TT + 4;                                  // row of wDt / wDu / wGy
-    static constexpr int PS = W + 4;                                   // row of the state partials
     static constexpr int XS = W * NS + 4;                              // row of the transpose
     static constexpr int kWdt = 0, kWdu = CPW * WS, kWgy = 2 * CPW * WS;
-    static constexpr int kWp = 3 * CPW * WS;                           // [3][NT][CPW][PS]
-    static constexpr int kWx = kWp + 3 * NT * CPW * PS;                // [32][XS]
+    static constexpr int kWx = 3 * CPW * WS;                           // [32][XS]
     static constexpr int WBUF = (kWx + 32 * XS) * 4;
     // dB/dC tile accumulator: [B or C][batch row][state][TT], rows rotated
     static constexpr int DBC_PAR = 2 * 2 * N * TT;
@@ -99,7 +97,7 @@ struct BwdLayout {
     static_assert(kAlloc <= 227 * 1024, "shared memory budget");
     static_assert(CPW * (TT / W) == 32, "one prep item of 8 steps per lane");
     static_assert(SSM_CKPT_CHUNK == W, "windows are checkpoint chunks");
-    static_assert(PS % 4 == 0 && WS % 4 == 0 && XS == 36 && TT == 32, "row shapes");
+    static_assert(WS % 4 == 0 && XS == 36 && TT == 32 && NT == 4 && W == 8, "row shapes");
 };
 
 // Column of step t of state n in the dB/dC accumulator.  The rotation puts
@@ -133,6 +131,20 @@ __device__ __forceinline__ float4 f4add(float4 a, float4 b) {
     return make_float4(lo.x, lo.y, hi.x, hi.y);
 }
 
+// Sum over the 4 state groups of a channel (lanes c, c+8, c+16, c+24) of the
+// partials of a 4-step half-window, held as (steps 0,1) and (steps 2,3):
+// two butterfly rounds (xor 16, then xor 8) leave lane group g with the
+// total of step g.
+__device__ __forceinline__ float group_reduce4(float2 p01, float2 p23, int g) {
+    const bool g1 = (g & 2) != 0, g0 = (g & 1) != 0;
+    float2 keep = g1 ? p23 : p01;
+    const float2 send = g1 ? p01 : p23;
+    keep.x += __shfl_xor_sync(0xffffffffu, send.x, 16);
+    keep.y += __shfl_xor_sync(0xffffffffu, send.y, 16);
+    const float k = g0 ? keep.y : keep.x, o = g0 ? keep.x : keep.y;
+    return k + __shfl_xor_sync(0xffffffffu, o, 8);
+}
+
 // ALN: the channel count is a multiple of 8 and CTAs and passes start on
 // multiples of 8 rows, so that no warp's 8 channels span two batch rows.
 template <typename T, int NWC, int STAGES, bool HZ, bool SP, bool ALN>
@@ -143,7 +155,7 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                const TmaBwdParams p) {
     using Ly = BwdLayout<T, NWC, STAGES>;
     constexpr int N = Ly::N, NT = Ly::NT, NS = Ly::NS, TT = Ly::TT, CPW = Ly::CPW;
-    constexpr int WS = Ly::WS, PS = Ly::PS, XS = Ly::XS, W = Ly::W;
+    constexpr int WS = Ly::WS, XS = Ly::XS, W = Ly::W;
 
     extern __shared__ __align__(128) uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -314,7 +326,7 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
     const int it_rl = lane / (TT / W), it_t = (lane % (TT / W)) * W;   // prep: row, step offset
     float *wbase = reinterpret_cast<float *>(smem + Ly::kW + warp * Ly::WBUF);
     float *wDt = wbase + Ly::kWdt, *wDu = wbase + Ly::kWdu, *wGy = wbase + Ly::kWgy;
-    float *wP = wbase + Ly::kWp, *wX = wbase + Ly::kWx;
+    float *wX = wbase + Ly::kWx;
     float *myX = wX + lane * XS;
 
     float2 A2p[NS], dA2[NS];                                   // (A log2 e) twice; dA partials
@@ -471,6 +483,9 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                 // Forward recompute over pairs of steps (f32x2 arithmetic):
                 // Ā_t, Ā_t h_{t-1}, the y partials and gy h_t (for dC).
                 float2 ab2[W / 2][NS], ahp2[W / 2][NS];
+                // per half-window, summed over the state groups: y, Σ λ A Ā h
+                // (units of A log2 e) and Σ λ B at step 4 hh + g of channel c
+                float yv[2], sav[2], sbv[2];
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     const int tb = tw + 4 * hh;
@@ -505,8 +520,7 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                         *reinterpret_cast<float4 *>(myX + (2 * j + hh) * 4) =
                             make_float4(xc[0].x, xc[0].y, xc[1].x, xc[1].y);
                     }
-                    *reinterpret_cast<float4 *>(wP + (0 * NT + g) * CPW * PS + c * PS + 4 * hh) =
-                        make_float4(y2[0].x, y2[0].y, y2[1].x, y2[1].y);
+                    yv[hh] = group_reduce4(y2[0], y2[1], g);
                 }
                 reduce_x(1, tw);
                 // Reverse sweep over pairs of steps.  The A-weighted sum is
@@ -546,51 +560,37 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                         *reinterpret_cast<float4 *>(myX + (2 * j + hh) * 4) =
                             make_float4(xb[0].x, xb[0].y, xb[1].x, xb[1].y);
                     }
-                    *reinterpret_cast<float4 *>(wP + (1 * NT + g) * CPW * PS + c * PS + 4 * hh) =
-                        make_float4(sa2[0].x, sa2[0].y, sa2[1].x, sa2[1].y);
-                    *reinterpret_cast<float4 *>(wP + (2 * NT + g) * CPW * PS + c * PS + 4 * hh) =
-                        make_float4(sb2[0].x, sb2[0].y, sb2[1].x, sb2[1].y);
+                    sav[hh] = group_reduce4(sa2[0], sa2[1], g);
+                    sbv[hh] = group_reduce4(sb2[0], sb2[1], g);
                 }
-                reduce_x(0, tw);   // its leading __syncwarp also publishes the partials
-                // per-element results: lane (g, c) finishes steps 2g and 2g+1 of channel c
-                if (live && tgw + 2 * g < p.L) {
-                    const int t = 2 * g;
-                    float2 y = make_float2(0.f, 0.f), a_sa = y, a_sb = y;
-#pragma unroll
-                    for (int gg = 0; gg < NT; ++gg) {
-                        y = __fadd2_rn(y, *reinterpret_cast<const float2 *>(wP + (0 * NT + gg) * CPW * PS + c * PS + t));
-                        a_sa = __fadd2_rn(a_sa, *reinterpret_cast<const float2 *>(wP + (1 * NT + gg) * CPW * PS + c * PS + t));
-                        a_sb = __fadd2_rn(a_sb, *reinterpret_cast<const float2 *>(wP + (2 * NT + gg) * CPW * PS + c * PS + t));
-                    }
-                    const int o = c * TT + tw + t;
-                    const float x[2] = {IO<T>::to_f(rawU[o]), IO<T>::to_f(rawU[o + 1])};
-                    const float gv[2] = {IO<T>::to_f(rawG[o]), IO<T>::to_f(rawG[o + 1])};
-                    const float2 dtv = *reinterpret_cast<const float2 *>(wDt + c * WS + tw + t);
-                    const float2 gyv = *reinterpret_cast<const float2 *>(wGy + c * WS + tw + t);
-                    const float yy[2] = {fmaf(Dd, x[0], y.x), fmaf(Dd, x[1], y.y)};
-                    const float sa2[2] = {a_sa.x * 0.69314718f, a_sa.y * 0.69314718f};
-                    const float sb2[2] = {a_sb.x, a_sb.y};
-                    const float dt2[2] = {dtv.x, dtv.y}, gy2[2] = {gyv.x, gyv.y};
-                    float dzv[2] = {0.f, 0.f}, duv[2], ddv[2];
+                reduce_x(0, tw);
+                // per-element results: lane (g, c) finishes steps g and g + 4 of channel c
+                if (live) {
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
+                        const int t = g + 4 * e;
+                        if (tgw + t >= p.L) continue;
+                        const int o = c * TT + tw + t;
+                        const float x = IO<T>::to_f(rawU[o]);
+                        const float gv = IO<T>::to_f(rawG[o]);
+                        const float dtv = wDt[c * WS + tw + t], gyv = wGy[c * WS + tw + t];
+                        const float yy = fmaf(Dd, x, yv[e]);
+                        const float sa = sav[e] * 0.69314718f, sb = sbv[e];
+                        const size_t off = (size_t)row * p.L + tgw + t;
                         if constexpr (HZ) {
-                            const float zz = IO<T>::to_f(rawZ[o + e]);
+                            const float zz = IO<T>::to_f(rawZ[o]);
                             const float sg = sigmoid(zz);
-                            dzv[e] = gv[e] * yy[e] * sg * fmaf(zz, 1.f - sg, 1.f);
+                            __stcs(p.dz + off, gv * yy * sg * fmaf(zz, 1.f - sg, 1.f));
                         }
-                        const float dDelta = fmaf(x[e], sb2[e], sa2[e]);
-                        ddv[e] = SP ? dDelta * sigmoid(IO<T>::to_f(rawD[o + e]) + bias_c) : dDelta;
-                        duv[e] = fmaf(gy2[e], Dd, dt2[e] * sb2[e]);
-                        dD_acc = fmaf(gy2[e], x[e], dD_acc);
-                        db_acc += ddv[e];
+                        const float dDelta = fmaf(x, sb, sa);
+                        const float ddv = SP ? dDelta * sigmoid(IO<T>::to_f(rawD[o]) + bias_c) : dDelta;
+                        __stcs(p.du + off, fmaf(gyv, Dd, dtv * sb));
+                        __stcs(p.ddelta + off, ddv);
+                        dD_acc = fmaf(gyv, x, dD_acc);
+                        db_acc += ddv;
                     }
-                    const size_t off = (size_t)row * p.L + tgw + t;
-                    __stcs(reinterpret_cast<float2 *>(p.du + off), make_float2(duv[0], duv[1]));
-                    __stcs(reinterpret_cast<float2 *>(p.ddelta + off), make_float2(ddv[0], ddv[1]));
-                    if constexpr (HZ) __stcs(reinterpret_cast<float2 *>(p.dz + off), make_float2(dzv[0], dzv[1]));
                 }
-                __syncwarp();   // wP and the transpose buffer are rewritten by the next window
+                __syncwarp();   // the transpose buffer is rewritten by the next window
             }
         }
         __syncwarp();
