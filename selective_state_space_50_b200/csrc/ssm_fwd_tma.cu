@@ -256,12 +256,14 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
 
     int s = 0, phase = 0;          // ring slot and its parity for tile kg
     int q = 0, tile = 0, q0 = 0, q1 = 0;
-    int rpw = CPW;                 // rows per warp in this pass (the same for every warp, +-1 row)
+    // Each warp takes a whole group of CPW rows of the pass (the last busy
+    // warp may hold fewer); warps past the pass's rows stay idle.  Fewer,
+    // fuller warps issue fewer instructions for the same rows than rows
+    // spread over every warp.
+    constexpr int rpw = CPW;
     for (int kg = 0; kg < total; ++kg) {
         if (tile == 0) {
             pass_rows(q, q0, q1);
-            // spread the pass's rows evenly over the warps
-            rpw = (q1 - q0 + NWC - 1) / NWC;
         }
         const int t0 = tile * TT;
         const int wrow0 = q0 + warp * rpw;   // first row of this warp in the pass
