@@ -154,7 +154,7 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                const __grid_constant__ CUtensorMap m_B, const __grid_constant__ CUtensorMap m_C,
                const TmaBwdParams p) {
     using Ly = BwdLayout<T, NWC, STAGES>;
-    constexpr int N = Ly::N, NT = Ly::NT, NS = Ly::NS, TT = Ly::TT, CPW = Ly::CPW;
+    constexpr int N = Ly::N, NS = Ly::NS, TT = Ly::TT, CPW = Ly::CPW;
     constexpr int WS = Ly::WS, XS = Ly::XS, W = Ly::W;
 
     extern __shared__ __align__(128) uint8_t smem_raw[];

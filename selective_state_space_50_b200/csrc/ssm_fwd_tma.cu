@@ -517,7 +517,10 @@ template <typename T, int N, int NT> struct TmaCfg;
     };
 using bf16_t = __nv_bfloat16;
 SSM_TMA_CFG(bf16_t, 16, 2, 9, SSM_TMA_STAGES)
-SSM_TMA_CFG(bf16_t, 16, 4, 12, SSM_TMA_STAGES)
+#ifndef SSM_TMA_NWC_BF16_N16
+#define SSM_TMA_NWC_BF16_N16 12
+#endif
+SSM_TMA_CFG(bf16_t, 16, 4, SSM_TMA_NWC_BF16_N16, SSM_TMA_STAGES)
 SSM_TMA_CFG(bf16_t, 16, 8, 12, 3)
 SSM_TMA_CFG(bf16_t, 16, 16, 7, 3)
 SSM_TMA_CFG(bf16_t, 32, 4, 12, SSM_TMA_STAGES)
