@@ -20,8 +20,8 @@
 //
 // Kernel: one 128 x 128 output tile per CTA, 4 warps.  Lane 0 of warp 0
 // streams 64-deep K slices of A and Bm into a shared-memory ring with TMA
-// (128-byte swizzle; 6 stages for x_proj, 1 for dt_proj whose K fits one
-// slice); lane 0 of warp 1 issues tcgen05.mma (M 128, N 128, K 16) on
+// (128-byte swizzle; 6 stages for x_proj, 1 or 3 for dt_proj whose K is one
+// to three slices); lane 0 of warp 1 issues tcgen05.mma (M 128, N 128, K 16) on
 // shared-memory descriptors and frees each stage with tcgen05.commit; warp 2
 // owns the tensor-memory allocation.  After the last commit all four warps
 // read the accumulator (warp w reads lanes 32w..32w+31, i.e. output rows),
@@ -57,7 +57,8 @@ static_assert(4 * kStgWarp <= kStage, "epilogue staging fits in one stage");
 // Shared memory of a STAGES-deep ring: the ring, then the barriers and the
 // tensor-memory address.  A one-stage kernel asks for at least 56 KB so that
 // at most four CTAs share an SM: four 128-column accumulators fill its 512
-// tensor-memory columns, and no allocation has to wait.
+// tensor-memory columns, and no allocation has to wait.  Deeper rings fit at
+// most two (3 stages) or one (6 stages) CTA per SM.
 template <int STAGES>
 struct ProjSmem {
     static constexpr int kBars = STAGES * kStage;
@@ -65,6 +66,7 @@ struct ProjSmem {
     static constexpr int kAlloc = kUsed > 56 * 1024 ? kUsed : 56 * 1024;
     static_assert(kAlloc <= 227 * 1024, "shared memory budget");
     static_assert(STAGES > 1 || 5 * kAlloc > 228 * 1024, "at most 4 one-stage CTAs per SM");
+    static_assert(STAGES == 1 || 3 * kAlloc > 228 * 1024, "at most 2 deeper-ring CTAs per SM");
 };
 
 struct ProjSeg {
@@ -287,13 +289,17 @@ cudaError_t launch_proj_gemm(const CUtensorMap &mA, const CUtensorMap &mB, const
     return cudaGetLastError();
 }
 
-// A deep ring when the contraction is long (x_proj streams the activations
-// through it); a single stage, with up to four CTAs per SM overlapping each
-// other's loads, MMAs and stores, when one K slice covers it (dt_proj).
+// Ring depth by contraction length.  One K slice (dt_proj at rank <= 64): a
+// single stage, with up to four CTAs per SM overlapping each other's loads,
+// MMAs and stores.  Two or three slices (larger ranks): the whole contraction
+// in flight at once, two CTAs per SM.  Longer (x_proj streams the
+// activations): a 6-stage ring.
 cudaError_t launch_proj_any(const CUtensorMap &mA, const CUtensorMap &mB, const ProjParams &p, int batch,
                             cudaStream_t stream) {
-    return p.K <= kBK ? launch_proj_gemm<1>(mA, mB, p, batch, stream)
-                      : launch_proj_gemm<6>(mA, mB, p, batch, stream);
+    const int nk = (p.K + kBK - 1) / kBK;
+    if (nk <= 1) return launch_proj_gemm<1>(mA, mB, p, batch, stream);
+    if (nk <= 3) return launch_proj_gemm<3>(mA, mB, p, batch, stream);
+    return launch_proj_gemm<6>(mA, mB, p, batch, stream);
 }
 
 }  // namespace
