@@ -39,11 +39,9 @@ namespace ssm {
 
 namespace {
 
-constexpr int kBM = 128, kBN = 128, kBK = 64;        // output tile, K slice
+constexpr int kBM = 128, kBK = 64;                    // output tile rows, K slice
 constexpr int kATile = kBM * kBK * 2;                 // [128 rows][64 k] bf16
 constexpr int kBChunk = kBK * 64 * 2;                 // [64 k][64 columns] bf16
-constexpr int kBTile = (kBN / 64) * kBChunk;
-constexpr int kStage = kATile + kBTile;
 constexpr int kThreads = 128;
 // Epilogue staging (reuses the ring): per warp 32 rows x 64 columns of bf16,
 // rows padded to 72 elements so that row-wise 16-byte writes spread over the
@@ -51,17 +49,28 @@ constexpr int kThreads = 128;
 constexpr int kStgRow = 72;
 constexpr int kStgWarp = 32 * kStgRow * 2;
 static_assert(kATile % 1024 == 0 && kBChunk % 1024 == 0, "swizzle atoms stay aligned");
-static_assert(kBN % 16 == 0 && kBN >= 16 && kBN <= 256, "UMMA N for M = 128");
-static_assert(4 * kStgWarp <= kStage, "epilogue staging fits in one stage");
+
+// An output tile of kBM x BN columns: the ring stage that feeds it and the
+// instruction descriptor of kind::f16 (fp32 accumulator, bf16 A and B,
+// A K-major, B N-major, N = BN, M = kBM).
+template <int BN>
+struct ProjTile {
+    static constexpr int kBTile = (BN / 64) * kBChunk;
+    static constexpr int kStage = kATile + kBTile;
+    static constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
+                                       ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
+    static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "whole 64-column chunks; UMMA N <= 256");
+    static_assert(4 * kStgWarp <= kStage, "epilogue staging fits in one stage");
+};
 
 // Shared memory of a STAGES-deep ring: the ring, then the barriers and the
 // tensor-memory address.  A one-stage kernel asks for at least 56 KB so that
 // at most four CTAs share an SM: four 128-column accumulators fill its 512
 // tensor-memory columns, and no allocation has to wait.  Deeper rings fit at
 // most two (3 stages) or one (6 stages) CTA per SM.
-template <int STAGES>
+template <int STAGES, int BN>
 struct ProjSmem {
-    static constexpr int kBars = STAGES * kStage;
+    static constexpr int kBars = STAGES * ProjTile<BN>::kStage;
     static constexpr int kUsed = kBars + (2 * STAGES + 1) * 8 + 16 + 1024;
     static constexpr int kAlloc = kUsed > 56 * 1024 ? kUsed : 56 * 1024;
     static_assert(kAlloc <= 227 * 1024, "shared memory budget");
@@ -110,18 +119,14 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t addr, uint32_t lbo, uint
            ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
 
-// Instruction descriptor of kind::f16: fp32 accumulator, bf16 A and B,
-// A K-major, B N-major, N = kBN, M = kBM.
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
-                            ((uint32_t)(kBN >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
-
-__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
     const uint32_t mask0 = 0, mask1 = 0, mask2 = 0, mask3 = 0;   // no output lanes disabled
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}"
-        ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate),
+        ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate),
           "r"(mask0), "r"(mask1), "r"(mask2), "r"(mask3)
         : "memory");
 }
@@ -149,13 +154,15 @@ __device__ __forceinline__ uint32_t pack_bf16x2(uint32_t lo, uint32_t hi) {
     return *reinterpret_cast<const uint32_t *>(&v);
 }
 
-template <int kStages>
+template <int kStages, int kBN>
 __global__ void __launch_bounds__(kThreads, 1)
 proj_gemm_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mB,
                  const ProjParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + ProjSmem<kStages>::kBars);
+    using Tile = ProjTile<kBN>;
+    constexpr int kStage = Tile::kStage;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + ProjSmem<kStages, kBN>::kBars);
     uint64_t *empty = full + kStages;
     uint64_t *accum = empty + kStages;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accum + 1);
@@ -217,7 +224,7 @@ proj_gemm_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__
                     //    (SBO), K step of 16 = 16 rows.
                     const uint64_t da = sw128_desc(a0 + kk * 32, 16, 1024);
                     const uint64_t db = sw128_desc(b0 + kk * 16 * 128, kBChunk, 1024);
-                    umma_bf16(tmem, da, db, (kt | kk) != 0);
+                    umma_bf16(tmem, da, db, Tile::kIdesc, (kt | kk) != 0);
                 }
                 umma_commit(empty + s);   // the stage is free once these MMAs are done
             }
@@ -274,20 +281,28 @@ proj_gemm_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__
     if (warp == 2) tmem_dealloc(tmem, kBN);
 }
 
-template <int STAGES>
+template <int STAGES, int BN>
 cudaError_t launch_proj_gemm(const CUtensorMap &mA, const CUtensorMap &mB, const ProjParams &p, int batch,
                              cudaStream_t stream) {
-    constexpr int smem = ProjSmem<STAGES>::kAlloc;
+    constexpr int smem = ProjSmem<STAGES, BN>::kAlloc;
     static bool attr_done = false;
     if (!attr_done) {
-        cudaError_t e = cudaFuncSetAttribute(proj_gemm_kernel<STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        cudaError_t e = cudaFuncSetAttribute(proj_gemm_kernel<STAGES, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         attr_done = true;
     }
-    const dim3 grid((unsigned)((p.L + kBN - 1) / kBN), (unsigned)((p.M + kBM - 1) / kBM), (unsigned)batch);
-    proj_gemm_kernel<STAGES><<<grid, kThreads, smem, stream>>>(mA, mB, p);
+    const dim3 grid((unsigned)((p.L + BN - 1) / BN), (unsigned)((p.M + kBM - 1) / kBM), (unsigned)batch);
+    proj_gemm_kernel<STAGES, BN><<<grid, kThreads, smem, stream>>>(mA, mB, p);
     return cudaGetLastError();
 }
+
+// Ring depth and tile width of the long contraction (x_proj).
+#ifndef SSM_PROJ_LONG_STAGES
+#define SSM_PROJ_LONG_STAGES 6
+#endif
+#ifndef SSM_PROJ_LONG_BN
+#define SSM_PROJ_LONG_BN 128
+#endif
 
 // Ring depth by contraction length.  One K slice (dt_proj at rank <= 64): a
 // single stage, with up to four CTAs per SM overlapping each other's loads,
@@ -297,9 +312,9 @@ cudaError_t launch_proj_gemm(const CUtensorMap &mA, const CUtensorMap &mB, const
 cudaError_t launch_proj_any(const CUtensorMap &mA, const CUtensorMap &mB, const ProjParams &p, int batch,
                             cudaStream_t stream) {
     const int nk = (p.K + kBK - 1) / kBK;
-    if (nk <= 1) return launch_proj_gemm<1>(mA, mB, p, batch, stream);
-    if (nk <= 3) return launch_proj_gemm<3>(mA, mB, p, batch, stream);
-    return launch_proj_gemm<6>(mA, mB, p, batch, stream);
+    if (nk <= 1) return launch_proj_gemm<1, 128>(mA, mB, p, batch, stream);
+    if (nk <= 3) return launch_proj_gemm<3, 128>(mA, mB, p, batch, stream);
+    return launch_proj_gemm<SSM_PROJ_LONG_STAGES, SSM_PROJ_LONG_BN>(mA, mB, p, batch, stream);
 }
 
 }  // namespace
