@@ -10,7 +10,8 @@
 //   dA = Σ λ Δ Ā h_{t-1},  dB = Σ_d λ Δ u,  dC = Σ_d gy h,  dD = Σ gy u,  dbias = Σ ddelta
 //
 // Organisation (mirrors the TMA forward):
-//  * One CTA per SM; channel rows (batch x dim) split evenly over the CTAs.
+//  * One CTA per SM; channel rows (batch x dim) split evenly over the CTAs, in
+//    units of 8 rows when dim is a multiple of 8.
 //    Time tiles of 32 steps are visited last to first.  A producer lane
 //    streams delta, u, z, dout ([rows x 32] boxes) and B, C ([dstate x 32]
 //    per batch row) into a two-stage ring with TMA loads that complete on
@@ -21,9 +22,10 @@
 //    the forward) from last to first, it starts from the checkpointed state,
 //    recomputes Ā_t (one ex2 per step and state) and Ā_t h_{t-1} into
 //    registers, and sweeps the window backwards carrying λ and Ā_{t+1}.
-//  * Sums over states for each (channel, step) -- y, Σ λ A Ā h, Σ λ B -- go
-//    through a per-warp buffer and are finished per element (dz, du, ddelta;
-//    dD and dbias accumulate per lane).  Sums over channels for each
+//  * Sums over states for each (channel, step) -- y, Σ λ A Ā h, Σ λ B -- are
+//    reduced over the channel's 4 state groups with warp shuffles, per 4-step
+//    half-window, and finished per element by the lane that holds the total
+//    (dz, du, ddelta; dD and dbias accumulate per lane).  Sums over channels for each
 //    (state, step) -- dB, dC -- are reduced over a quarter-warp's 8 channels
 //    by a transpose through shared memory, accumulated over the CTA's warps
 //    with shared-memory atomics into a per-tile buffer, and flushed by the

@@ -12,7 +12,8 @@
 //    z (a [rows x TT] box each) and B, C (a [dstate x TT] box per batch row)
 //    into a STAGES-deep shared-memory ring with 2-D TMA loads completing on
 //    mbarriers.
-//  * Consumer warps own 32/NT channels each; lane (c, g) owns NS = N/NT
+//  * Consumer warps own 32/NT channels each (whole groups of rows; warps past
+//    a pass's rows stay idle); lane (c, g) owns NS = N/NT
 //    states of channel c and keeps them in fp32 registers for the whole
 //    sequence.  Per tile a warp (1) computes Δ and Δ·u once per element into
 //    a warp-private fp32 buffer, (2) runs the recurrence, two time steps per
