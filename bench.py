@@ -176,7 +176,7 @@ def aggregate_rate(world: int, steps: int, units_per_step: int, t_dev_s: float) 
     return world * steps * units_per_step / max_over_ranks(t_dev_s, world)
 
 
-def cpu_oracle_rate(w, inp, budget_s: float, nthreads: int = 0):
+def cpu_oracle_rate(w, inp, budget_s: float, nthreads: int = 0, zoh: bool = False):
     """Times the fp64 oracle on whole-batch channel slices until about
     `budget_s` seconds of wall time are spent.  Returns (elem/s, threads, desc)."""
     import oracle
@@ -194,7 +194,7 @@ def cpu_oracle_rate(w, inp, budget_s: float, nthreads: int = 0):
         t = time.perf_counter()
         oracle.fwd(sub["u_f64"], sub["delta_f64"], sub["A_f64"], sub["B_f64"], sub["C_f64"],
                    sub["D_f64"], sub["z_f64"], sub["delta_bias_f64"], w.softplus,
-                   nthreads=nthreads)
+                   zoh=zoh, nthreads=nthreads)
         t_total += time.perf_counter() - t
         done_elems += w.batch * step * w.seqlen
         slices += 1
@@ -366,7 +366,7 @@ def run_ours(args, world, rank, local):
     else:
         def fwd():
             ssm_scan.fwd_raw(shape, dv["u"], dv["delta"], dv["A"], dv["B"], dv["C"], dv["D"],
-                             dv["z"], dv["delta_bias"], True, out, last, None, stream)
+                             dv["z"], dv["delta_bias"], True, out, last, None, stream, zoh=args.zoh)
 
     for _ in range(max(3, args.warmup)):
         flush.zero_()
@@ -448,7 +448,7 @@ def run_ours(args, world, rank, local):
         o, _, ckp = ssm_scan.selective_scan_fwd(dtmp["u"], dtmp["delta"], dtmp["A"], dtmp["B"],
                                                 dtmp["C"], dtmp["D"], dtmp["z"], dtmp["delta_bias"],
                                                 True, return_last_state=True, out=out,
-                                                return_ckpt=fwdbwd)
+                                                return_ckpt=fwdbwd, zoh=args.zoh)
         if fwdbwd:
             g = ssm_scan.selective_scan_bwd(dtmp["u"], dtmp["delta"], dtmp["A"], dtmp["B"],
                                             dtmp["C"], dtmp["D"], dtmp["z"], dtmp["delta_bias"],
@@ -510,6 +510,8 @@ def run_ours(args, world, rank, local):
         "gpu_launches": args.steps * (3 if proj else 2 if fwdbwd else
                                       (3 * args.segments if args.segments > 1 else 1)),
     }
+    if args.zoh:
+        line["config"]["discretization"] = "zero-order hold"
     if seg_info:
         line["segments"] = seg_info
         line["config"]["step"] = (f"sequence cut into {args.segments} segments: pass 1 over all, "
@@ -525,7 +527,7 @@ def run_ours(args, world, rank, local):
                                        "frac": pb / t_proj / 1e9 / float(peaks["hbm_gbs"])},
                                "tflops": flops / t_proj / 1e12}
     if world == 1 and not args.no_cpu_baseline:
-        rate, cores, desc = cpu_oracle_rate(w, inp, args.cpu_budget)
+        rate, cores, desc = cpu_oracle_rate(w, inp, args.cpu_budget, zoh=args.zoh)
         if proj:
             # the oracle's projections on one batch row x 256 steps (all channels)
             import oracle
@@ -669,6 +671,8 @@ def main():
                     help="workload to time (default: the Mamba-130M layer shape)")
     ap.add_argument("--seqlen", type=int, default=0,
                     help="override the workload's sequence length (for profiling small cases)")
+    ap.add_argument("--zoh", action="store_true",
+                    help="zero-order-hold discretisation (forward workloads)")
     ap.add_argument("--segments", type=int, default=1,
                     help="run the forward as S sequence segments with the sharded protocol")
     ap.add_argument("--decode", action="store_true",
