@@ -145,8 +145,39 @@ __device__ __forceinline__ void load_pairs8_at<float>(const float *lo, const flo
     v[2] = make_float2(b.x, b.y); v[3] = make_float2(b.z, b.w);
 }
 
-// FL < 0: the gate, softplus and checkpoint options are read at run time;
-// otherwise they are compile-time bits (1: gate z, 2: softplus, 4: checkpoints).
+// Zero-order-hold factor φ = (Ā - 1)/(Δ A) for a pair of steps of one state,
+// with arg = Δ A log2(e), a = 2^arg = Ā, idt = 1/Δ per step and ia = 1/A:
+// (a - 1) · idt · ia, or, for |Δ A| < 0.1 where a - 1 cancels, the Taylor
+// series 1 + x/2 + x²/6 + x³/24 + x⁴/120 + x⁵/720 in x = arg ln 2 (its
+// coefficients below are pre-scaled by powers of ln 2, so it runs in arg).
+// Exact zeros (Δ = 0 or A = 0) take the series: φ = 1, the Δ·B limit.
+__device__ __forceinline__ float2 zoh_phi2(float2 arg, float2 a, float2 idt, float2 ia) {
+    constexpr float L1 = 0.34657359f;      // ln2 / 2
+    constexpr float L2 = 0.080075108f;     // ln2^2 / 6
+    constexpr float L3 = 0.013874226f;     // ln2^3 / 24
+    constexpr float L4 = 0.0019234117f;    // ln2^4 / 120
+    constexpr float L5 = 0.00022220567f;   // ln2^5 / 720
+    float2 ser = __ffma2_rn(arg, make_float2(L5, L5), make_float2(L4, L4));
+    ser = __ffma2_rn(arg, ser, make_float2(L3, L3));
+    ser = __ffma2_rn(arg, ser, make_float2(L2, L2));
+    ser = __ffma2_rn(arg, ser, make_float2(L1, L1));
+    ser = __ffma2_rn(arg, ser, make_float2(1.f, 1.f));
+    const float2 em1 = __fadd2_rn(a, make_float2(-1.f, -1.f));
+    const float2 q = __fmul2_rn(__fmul2_rn(em1, idt), ia);
+    constexpr float kSmall = 0.14426950f;  // |Δ A| < 0.1  <=>  |arg| < 0.1 log2(e)
+    return make_float2(fabsf(arg.x) < kSmall ? ser.x : q.x, fabsf(arg.y) < kSmall ? ser.y : q.y);
+}
+
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// FL >= 0: the gate, softplus and checkpoint options are compile-time bits
+// (1: gate z, 2: softplus, 4: checkpoints); B̄ = Δ B.  FL = -1: the options
+// are read at run time; B̄ = Δ B.  FL = -2: options at run time, zero-order
+// hold B̄ = φ(Δ A) Δ B.
 template <typename T, int NT, int NS, int TT, int NWC, int STAGES, int FL>
 __global__ void __launch_bounds__((NWC + 1) * 32, 1)
 fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constant__ CUtensorMap m_u,
@@ -156,6 +187,7 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
     constexpr int N = Ly::N, CPW = Ly::CPW, WS = Ly::WS, CHUNK = Ly::CHUNK;
     constexpr int IPL = Ly::ITEMS / 32;   // prep/epilogue items per lane
     constexpr int CPR = TT / CHUNK;       // chunks per row
+    constexpr bool ZOH = FL == -2;
     const bool has_z = FL < 0 ? p.has_z != 0 : (FL & 1) != 0;
     const bool softplus = FL < 0 ? p.softplus != 0 : (FL & 2) != 0;
     float *const ckpt = (FL < 0 || (FL & 4)) ? p.ckpt : nullptr;
@@ -247,6 +279,7 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
     float *wY = wDu + CPW * WS;      // [NT][CPW][WS] readout partials
 
     float2 A2d[NS];                  // A[d, n] log2(e), duplicated for f32x2 math
+    float2 iAd[NS];                  // 1 / A[d, n], duplicated (zero-order hold only)
     float h[NS];
     bool poly_ok = false;            // every A of this warp <= 0 (ex2_poly2 applies)
     int bsel = 0;
@@ -277,8 +310,13 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
             bool neg = true;
 #pragma unroll
             for (int j = 0; j < NS; ++j) {
-                const float a = live ? p.A[(size_t)d * N + g * NS + j] * SSM_LOG2E : 0.f;
+                const float av = live ? p.A[(size_t)d * N + g * NS + j] : 0.f;
+                const float a = av * SSM_LOG2E;
                 A2d[j] = make_float2(a, a);
+                if constexpr (ZOH) {
+                    const float ia = 1.f / av;
+                    iAd[j] = make_float2(ia, ia);
+                }
                 h[j] = (live && p.h0) ? p.h0[(size_t)row * N + g * NS + j] : 0.f;
                 neg = neg && a <= 0.f;
             }
@@ -371,6 +409,12 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                         dup[0] = make_float2(e.x, e.y); dup[1] = make_float2(e.z, e.w);
                         dup[2] = make_float2(f.x, f.y); dup[3] = make_float2(f.z, f.w);
                     }
+                    float2 idt[4];           // 1/Δ per step (zero-order hold only)
+                    if constexpr (ZOH) {
+#pragma unroll
+                        for (int pp = 0; pp < 4; ++pp)
+                            idt[pp] = make_float2(rcp_approx(dtp[pp].x), rcp_approx(dtp[pp].y));
+                    }
                     float2 y2[4];
 #pragma unroll
                     for (int pp = 0; pp < 4; ++pp) y2[pp] = make_float2(0.f, 0.f);
@@ -388,7 +432,8 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                             } else {
                                 a = make_float2(ex2(arg.x), ex2(arg.y));
                             }
-                            const float2 beta = __fmul2_rn(dup[pp], bq[pp]);
+                            float2 beta = __fmul2_rn(dup[pp], bq[pp]);
+                            if constexpr (ZOH) beta = __fmul2_rn(beta, zoh_phi2(arg, a, idt[pp], iAd[j]));
                             const float h0 = fmaf(a.x, h[j], beta.x);
                             const float h1 = fmaf(a.y, h0, beta.y);
                             h[j] = h1;
@@ -545,6 +590,9 @@ SSM_TMA_CFG(float, 8, 8, 8, 2)
 template <typename T, int N, int NT>
 cudaError_t launch_nt(const FwdParams &fp, cudaStream_t stream) {
     using C = TmaCfg<T, N, NT>;
+    if constexpr (N == 16) {   // zero-order hold: dstate 16 only (else the general kernel)
+        if (fp.zoh) return launch_cfg<T, NT, N / NT, C::TT, C::NWC, C::STAGES, -2>(fp, stream);
+    }
     // the benchmarked bf16 dstate-16 splits get compile-time options for the
     // usual combinations (gate and softplus on, with or without checkpoints)
     if constexpr (sizeof(T) == 2 && N == 16 && (NT == 2 || NT == 4 || NT == 16)) {
@@ -597,7 +645,7 @@ bool nt_valid(int N, int nt) {
 // Returns true (and launches) when the TMA path applies; false means the
 // caller should use the general kernel.
 bool try_launch_fwd_tma(const FwdParams &fp, cudaStream_t stream, cudaError_t *err) {
-    if (!fp.vec_ok || !fp.out || fp.zoh) return false;   // zero-order hold: general kernel
+    if (!fp.vec_ok || !fp.out || (fp.zoh && fp.N != 16)) return false;   // ZOH: dstate 16 here
     if (fp.N != 8 && fp.N != 16 && fp.N != 32) return false;
     if (!tma_available()) return false;
     const long long P = (long long)fp.batch * fp.dim;

@@ -47,6 +47,8 @@ CASES = [
     (2, 17, 64, 32, "f32", True, True, True, True, "neg_lognormal"),
     (1, 70, 100, 2, "bf16", True, True, True, True, "neg_lognormal"),
     (2, 1200, 64, 16, "bf16", True, True, True, True, "neg_lognormal"),   # shape of the TMA kernels
+    (2, 2400, 72, 16, "f32", True, True, True, True, "neg_lognormal"),    # TMA forward, ragged tile
+    (1, 4800, 264, 16, "bf16", False, True, True, True, "neg_n1"),        # TMA forward, no gate
 ]
 
 
