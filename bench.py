@@ -300,14 +300,14 @@ def run_ours(args, world, rank, local):
             # one training step of the scan: forward keeping checkpoints, backward
             if not bwd_only:
                 ssm_scan.fwd_raw(shape, dv["u"], dv["delta"], dv["A"], dv["B"], dv["C"], dv["D"],
-                                 dv["z"], dv["delta_bias"], True, out, last, ck, stream)
+                                 dv["z"], dv["delta_bias"], True, out, last, ck, stream, zoh=args.zoh)
             ssm_scan.bwd_raw(shape, dv["u"], dv["delta"], dv["A"], dv["B"], dv["C"], dv["D"],
                              dv["z"], dv["delta_bias"], True, dv["dout"], ck, grads["du"],
                              grads["ddelta"], grads["dA"], grads["dB"], grads["dC"], grads["dD"],
-                             grads["dz"], grads["ddelta_bias"], None, stream)
+                             grads["dz"], grads["ddelta_bias"], None, stream, zoh=args.zoh)
         if bwd_only:   # checkpoints for the timed backward-only steps
             ssm_scan.fwd_raw(shape, dv["u"], dv["delta"], dv["A"], dv["B"], dv["C"], dv["D"],
-                             dv["z"], dv["delta_bias"], True, out, last, ck, stream)
+                             dv["z"], dv["delta_bias"], True, out, last, ck, stream, zoh=args.zoh)
     elif args.segments > 1:
         # the sequence cut into S segments, run with the sharded protocol on
         # this one GPU (pass 1 over all segments, combine, pass 2 over 1..S-1)
@@ -452,7 +452,7 @@ def run_ours(args, world, rank, local):
         if fwdbwd:
             g = ssm_scan.selective_scan_bwd(dtmp["u"], dtmp["delta"], dtmp["A"], dtmp["B"],
                                             dtmp["C"], dtmp["D"], dtmp["z"], dtmp["delta_bias"],
-                                            True, dtmp["dout"], ckpt=ckp)
+                                            True, dtmp["dout"], ckpt=ckp, zoh=args.zoh)
             du_h.copy_(g["du"], non_blocking=True)
         out_h.copy_(o, non_blocking=True)
     for _ in range(3):
