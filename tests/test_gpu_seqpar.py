@@ -83,6 +83,7 @@ SHARD_CASES = [
     (2, 2400, 256, 16, "bf16", 2),
     (1, 4800, 1024, 16, "bf16", 8),
     (2, 64, 96, 16, "f32", 3),
+    (8, 1536, 256, 16, "bf16", 2),        # 4 lanes per channel (the layer shape's split)
 ]
 
 
