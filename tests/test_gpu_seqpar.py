@@ -41,6 +41,7 @@ SEG_CASES = [
     (1, 4800, 256, 16, "bf16", False),    # TMA kernel, one batch row
     (2, 64, 100, 16, "f32", False),       # general kernel
     (2, 40, 64, 8, "f32", True),          # general kernel, zero-order hold
+    (2, 2400, 72, 16, "bf16", True),      # TMA kernel, zero-order hold
 ]
 
 
