@@ -191,6 +191,7 @@ ssm_status_t fwd_impl(const ssm_shape_t *shape, const ssm_options_t *opts, const
     ssm::FwdParams p{};
     p.u = u; p.delta = delta; p.A = A; p.B = B; p.C = C; p.D = D; p.z = z;
     p.delta_bias = delta_bias; p.out = out; p.last_state = last_state; p.ckpt = ckpt; p.h0 = h0;
+    p.delta_sum = delta_sum;
     p.batch = shape->batch; p.dim = shape->dim; p.L = shape->seqlen; p.N = shape->dstate;
     p.n_ckpt = n_ckpt(shape);
     p.softplus = opts->delta_softplus != 0;
@@ -200,10 +201,6 @@ ssm_status_t fwd_impl(const ssm_shape_t *shape, const ssm_options_t *opts, const
                aligned16(B) && aligned16(C) && aligned16(out) && (!z || aligned16(z));
     cudaError_t e = ssm::launch_fwd(p, false, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "ssm_selective_scan_fwd launch");
-    if (delta_sum) {
-        e = ssm::launch_delta_sum(p, delta_sum, static_cast<cudaStream_t>(stream));
-        if (e != cudaSuccess) return cuda_fail(e, "ssm_selective_scan_fwd_segment delta sums");
-    }
     return ok();
 }
 

@@ -307,13 +307,17 @@ cudaError_t launch_fwd(const FwdParams &p, bool states_only, cudaStream_t stream
     const FwdKernel choice = fwd_kernel_choice();
     if (!states_only && choice != FwdKernel::kGeneral) {
         cudaError_t e = cudaSuccess;
-        if (try_launch_fwd_tma(p, stream, &e)) return e;
+        if (try_launch_fwd_tma(p, stream, &e)) return e;   // also writes delta_sum
         if (choice == FwdKernel::kTma) return cudaErrorNotSupported;
     }
+    cudaError_t e;
     if (p.io_bf16)
-        return states_only ? launch_fwd_t<__nv_bfloat16, 1>(p, stream)
-                           : launch_fwd_t<__nv_bfloat16, 0>(p, stream);
-    return states_only ? launch_fwd_t<float, 1>(p, stream) : launch_fwd_t<float, 0>(p, stream);
+        e = states_only ? launch_fwd_t<__nv_bfloat16, 1>(p, stream)
+                        : launch_fwd_t<__nv_bfloat16, 0>(p, stream);
+    else
+        e = states_only ? launch_fwd_t<float, 1>(p, stream) : launch_fwd_t<float, 0>(p, stream);
+    if (e == cudaSuccess && p.delta_sum) e = launch_delta_sum(p, p.delta_sum, stream);
+    return e;
 }
 
 }  // namespace ssm

@@ -62,6 +62,7 @@ constexpr int align128(int x) { return (x + 127) / 128 * 128; }
 struct TmaFwdParams {
     const float *A, *D, *delta_bias;
     const float *h0;    // [P][N] state before step 0; NULL: zeros
+    float *delta_sum;   // [P] Σ_t Δ_t of each row, or NULL
     void *out;
     float *last_state, *ckpt;
     int P;          // batch * dim channel rows
@@ -286,6 +287,7 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
     bool live = false;
     // per-item constants for the prep / epilogue rows
     float Dd[IPL], bias[IPL];
+    float dsum[IPL];                 // Σ Δ of this lane's prep items over the pass (delta_sum)
     int irow[IPL];
 
     int s = 0, phase = 0;          // ring slot and its parity for tile kg
@@ -327,6 +329,7 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                 const bool ok = rr < wend;
                 const int dd = ok ? rr % p.dim : 0;
                 irow[i] = ok ? rr : -1;
+                dsum[i] = 0.f;
                 Dd[i] = (ok && p.D) ? p.D[dd] : 0.f;
                 bias[i] = (ok && p.delta_bias) ? p.delta_bias[dd] : 0.f;
             }
@@ -366,6 +369,11 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                         dt[v0 + k] = d2.x; dt[v0 + k + 1] = d2.y;
                         du[v0 + k] = u2.x; du[v0 + k + 1] = u2.y;
                     }
+                }
+#pragma unroll
+                if (p.delta_sum) {
+#pragma unroll
+                    for (int k = 0; k < CHUNK; ++k) dsum[i] += dt[k];
                 }
 #pragma unroll
                 for (int k = 0; k < CHUNK; k += 4) {
@@ -508,6 +516,17 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
         __syncwarp();
         if (lane == 0) mbar_arrive(empty + s);
         if (++s == STAGES) { s = 0; phase ^= 1; }
+        if (tile == ntiles - 1 && p.delta_sum && wrow0 < wend) {
+            // end of the pass: the CPR lanes holding a row's chunks (consecutive
+            // lanes of one item index) sum their shares; the first one stores
+#pragma unroll
+            for (int i = 0; i < IPL; ++i) {
+                float v = dsum[i];
+#pragma unroll
+                for (int m = 1; m < CPR; m <<= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
+                if (irow[i] >= 0 && (lane % CPR) == 0) p.delta_sum[irow[i]] = v;
+            }
+        }
         if (++tile == ntiles) { tile = 0; ++q; }
     }
 }
@@ -533,7 +552,7 @@ cudaError_t launch_cfg(const FwdParams &fp, cudaStream_t stream) {
         return cudaErrorInvalidValue;
     TmaFwdParams p{};
     p.A = fp.A; p.D = fp.D; p.delta_bias = fp.delta_bias; p.out = fp.out;
-    p.last_state = fp.last_state; p.ckpt = fp.ckpt; p.h0 = fp.h0;
+    p.last_state = fp.last_state; p.ckpt = fp.ckpt; p.h0 = fp.h0; p.delta_sum = fp.delta_sum;
     p.P = P; p.dim = fp.dim; p.L = fp.L; p.n_ckpt = fp.n_ckpt;
     p.softplus = fp.softplus; p.has_z = fp.z != nullptr; p.rows_max = rows_max;
     p.err = device_error_word();

@@ -19,6 +19,7 @@ struct FwdParams {
     void *out;
     float *last_state, *ckpt;
     const float *h0;  // [batch][dim][N] state before step 0; NULL: zeros
+    float *delta_sum; // [batch][dim] Σ_t Δ_t, or NULL (sequence segments)
     int batch, dim, L, N, n_ckpt;
     int softplus;
     int zoh;      // zero-order-hold B̄ (general kernels only)

@@ -10,7 +10,9 @@
 // exp(A Σ Δ_s) h_in(s) + e_s.
 //
 //  * delta_sum_kernel: Σ_t Δ_t per (batch, channel) of one segment, with the
-//    scan's own Δ = softplus(delta + bias) (one warp per channel row).
+//    scan's own Δ = softplus(delta + bias) (one warp per channel row), after
+//    the general forward kernel.  The TMA forward sums Δ itself, in the same
+//    pass that forms it.
 //  * combine_kernel: the exclusive scan of the summaries across segments,
 //    one thread per (channel row, state).
 
