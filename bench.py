@@ -255,6 +255,7 @@ def run_reference(args, world, rank):
 def run_ours(args, world, rank, local):
     import torch
     from selective_state_space_50_b200 import ssm_scan
+    from selective_state_space_50_b200 import dp
     from selective_state_space_50_b200.workloads import WORKLOADS, generate, to_torch
 
     proj = args.workload in PROJ_WORKLOADS
@@ -305,6 +306,10 @@ def run_ours(args, world, rank, local):
                              dv["z"], dv["delta_bias"], True, dv["dout"], ck, grads["du"],
                              grads["ddelta"], grads["dA"], grads["dB"], grads["dC"], grads["dD"],
                              grads["dz"], grads["ddelta_bias"], None, stream, zoh=args.zoh)
+            if world > 1:
+                # data parallel: the ranks hold batch rows of one layer, so the
+                # parameter gradients are summed over ranks (NCCL all-reduce)
+                dp.allreduce_param_grads(grads)
         if bwd_only:   # checkpoints for the timed backward-only steps
             ssm_scan.fwd_raw(shape, dv["u"], dv["delta"], dv["A"], dv["B"], dv["C"], dv["D"],
                              dv["z"], dv["delta_bias"], True, out, last, ck, stream, zoh=args.zoh)
@@ -494,7 +499,9 @@ def run_ours(args, world, rank, local):
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "dim": w.dim,
                    "dstate": w.dstate, "io_dtype": w.io_dtype, "state_dtype": "f32",
-                   "parallelism": f"replicas x{world} (independent batches)",
+                   "parallelism": (f"data parallel x{world} (own batch rows per rank; parameter "
+                                   f"gradients all-reduced)" if fwdbwd and world > 1 else
+                                   f"replicas x{world} (independent batches)"),
                    "l2": "flushed between steps (256 MiB write, outside the timed events)"},
         "gbs": alg_bytes / mean_s / 1e9,
         "roofline": {"bound": "alu", "achieved": achieved / 1e12, "peak": mufu_peak / 1e12,

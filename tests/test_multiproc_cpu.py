@@ -143,3 +143,39 @@ def test_sequence_sharded_forward_protocol_gloo(world):
         assert ok_out and ok_last, rank
         # pass 1 from zeros everywhere; pass 2 from the carry-in on ranks > 0 only
         assert calls == ([False] if rank == 0 else [False, True])
+
+
+def _dp_worker(rank, world, port, out_q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import torch
+    import torch.distributed as dist
+
+    from selective_state_space_50_b200 import dp
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        g = {"dA": torch.full((6, 4), float(rank + 1)), "dD": torch.arange(6.0) * (rank + 1),
+             "ddelta_bias": None, "du": torch.full((2, 6, 8), float(rank))}
+        dp.allreduce_param_grads(g)
+        tot = sum(r + 1 for r in range(world))
+        ok = (torch.equal(g["dA"], torch.full((6, 4), float(tot)))
+              and torch.equal(g["dD"], torch.arange(6.0) * tot)
+              and g["ddelta_bias"] is None
+              and torch.equal(g["du"], torch.full((2, 6, 8), float(rank))))   # activation grads untouched
+        out_q.put((rank, bool(ok)))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_data_parallel_param_grad_allreduce_gloo():
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_dp_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(world))
+    assert all(ok for _, ok in res)
