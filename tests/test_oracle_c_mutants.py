@@ -71,10 +71,14 @@ def _fails(pins):
 
 
 @pytest.fixture(scope="module")
-def built_mutants(tmp_path_factory):
+def built_mutants():
+    import pathlib
     src = open(SRC).read()
     out = {}
-    d = tmp_path_factory.mktemp("oracle_mutants")
+    # a scratch folder inside the repository's (git-ignored) build area
+    d = pathlib.Path(os.path.dirname(os.path.dirname(os.path.abspath(__file__)))) / "_build" / "oracle_mutants"
+    shutil.rmtree(d, ignore_errors=True)
+    d.mkdir(parents=True)
     for i, (name, (old, new)) in enumerate(MUTANTS.items()):
         assert src.count(old) == 1, name
         msrc = d / f"m{i}.c"
