@@ -131,9 +131,10 @@ ssm_status_t ssm_selective_scan_fwd(const ssm_shape_t *shape,
 
 /*
  * ssm_selective_scan_fwd with options: opts->delta_softplus replaces
- * delta_softplus and opts->discretization selects B̄ (SSM_DISC_ZOH is served
- * by the general kernel).  Checkpoints written with SSM_DISC_ZOH must be
- * passed to a backward with SSM_DISC_ZOH.
+ * delta_softplus and opts->discretization selects B̄ (the backward serves
+ * SSM_DISC_ZOH with its general kernel; the forward with its fast kernel at
+ * dstate 16).  Checkpoints written with SSM_DISC_ZOH must be passed to a
+ * backward with SSM_DISC_ZOH.
  * Errors: as ssm_selective_scan_fwd, plus SSM_ERR_INVALID_ARG for a NULL
  * opts or an unknown discretization.
  */
