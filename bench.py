@@ -687,6 +687,11 @@ def main():
     ap.add_argument("--decode", action="store_true",
                     help="time the single-step recurrent update instead of the scan")
     args = ap.parse_args()
+    if args.zoh and (args.decode or args.segments > 1 or args.workload in PROJ_WORKLOADS):
+        ap.error("--zoh applies to the scan workloads (not --decode, --segments or the projections)")
+    if args.segments > 1 and (args.decode or args.workload in PROJ_WORKLOADS
+                              or args.workload.endswith("fwdbwd")):
+        ap.error("--segments applies to the forward scan workloads")
     world, rank, local = dist_setup(args)
     try:
         if args.impl == "reference":
