@@ -66,6 +66,20 @@ def forward_segments(run_segment: Callable[[int, Optional[object]], Tuple], nseg
 
 # ---------------------------------------------------------------- CUDA + NCCL
 
+def all_gather_stacked(x, group=None):
+    """x of every rank of `group`, stacked in rank order: [world, *x.shape].
+    One all_gather_into_tensor into a buffer of the concatenated form (rank
+    blocks along the first dimension), which every backend accepts."""
+    import torch
+    import torch.distributed as dist
+    world = dist.get_world_size(group)
+    x = x.contiguous()
+    flat = x.reshape(-1)
+    buf = torch.empty(world * flat.numel(), device=x.device, dtype=x.dtype)
+    dist.all_gather_into_tensor(buf, flat, group=group)
+    return buf.view((world,) + tuple(x.shape))
+
+
 def cuda_forward_rank(u, delta, A, B, C, D=None, z=None, delta_bias=None,
                       delta_softplus: bool = True, group=None, stream=None):
     """Sequence-sharded forward on this rank's GPU: u, delta, z [batch, dim,
@@ -73,11 +87,9 @@ def cuda_forward_rank(u, delta, A, B, C, D=None, z=None, delta_bias=None,
     rank order make up the sequence).  The exchange is an all-gather on the
     torch.distributed group (NCCL for CUDA tensors).  Returns (out,
     last_state) of this segment."""
-    import torch
     import torch.distributed as dist
 
     from . import ssm_scan
-    world = dist.get_world_size(group)
     rank = dist.get_rank(group)
 
     def run_segment(h0):
@@ -85,10 +97,7 @@ def cuda_forward_rank(u, delta, A, B, C, D=None, z=None, delta_bias=None,
                                                    delta_softplus, h0=h0, stream=stream)
 
     def gather(x):
-        x = x.contiguous()
-        buf = torch.empty((world,) + tuple(x.shape), device=x.device, dtype=x.dtype)
-        dist.all_gather_into_tensor(buf, x, group=group)
-        return buf
+        return all_gather_stacked(x, group)
 
     def combine(dsums, ends):
         return ssm_scan.combine_carries(A, dsums, ends, stream=stream)

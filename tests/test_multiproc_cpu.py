@@ -110,10 +110,8 @@ def _seqpar_worker(rank, world, port, out_q):
                                    z[..., sl], bias, True, h0=None if h0 is None else h0.numpy())
             return out, torch.from_numpy(last), torch.from_numpy(oracle.delta_sums(delta[..., sl], bias))
 
-        def gather(x):
-            parts = [torch.empty_like(x) for _ in range(world)]
-            dist.all_gather(parts, x)
-            return torch.stack(parts)
+        def gather(x):   # the helper the CUDA path uses, here over gloo
+            return seqpar.all_gather_stacked(x)
 
         def combine(ds, es):
             return torch.from_numpy(oracle.combine_carries(A, ds.numpy(), es.numpy()))
