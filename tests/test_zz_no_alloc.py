@@ -11,7 +11,6 @@ passes on its own in a fresh process.
 """
 import ctypes
 
-import numpy as np
 import pytest
 import torch
 
