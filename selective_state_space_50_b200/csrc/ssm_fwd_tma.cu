@@ -154,10 +154,10 @@ __device__ __forceinline__ void load_pairs8_at<float>(const float *lo, const flo
 // Exact zeros (Δ = 0 or A = 0) take the series: φ = 1, the Δ·B limit.
 __device__ __forceinline__ float2 zoh_phi2(float2 arg, float2 a, float2 idt, float2 ia) {
     constexpr float L1 = 0.34657359f;      // ln2 / 2
-    constexpr float L2 = 0.080075108f;     // ln2^2 / 6
-    constexpr float L3 = 0.013874226f;     // ln2^3 / 24
-    constexpr float L4 = 0.0019234117f;    // ln2^4 / 120
-    constexpr float L5 = 0.00022220567f;   // ln2^5 / 720
+    constexpr float L2 = 0.080075502f;     // ln2^2 / 6
+    constexpr float L3 = 0.013876027f;     // ln2^3 / 24
+    constexpr float L4 = 0.0019236258f;    // ln2^4 / 120
+    constexpr float L5 = 0.00022222597f;   // ln2^5 / 720
     float2 ser = __ffma2_rn(arg, make_float2(L5, L5), make_float2(L4, L4));
     ser = __ffma2_rn(arg, ser, make_float2(L3, L3));
     ser = __ffma2_rn(arg, ser, make_float2(L2, L2));

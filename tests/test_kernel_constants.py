@@ -1,0 +1,42 @@
+"""Constants written into the CUDA sources, checked on the CPU against the
+mathematics they come from (their use is covered by the GPU parity tests;
+these catch a mistyped digit before a GPU run)."""
+import math
+import os
+import re
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+CSRC = os.path.join(ROOT, "selective_state_space_50_b200", "csrc")
+
+
+def _consts(path, names):
+    src = open(os.path.join(CSRC, path)).read()
+    out = {}
+    for n in names:
+        m = re.search(r"constexpr float " + n + r" = ([0-9.eE+-]+)f;", src)
+        assert m, n
+        out[n] = float(m.group(1))
+    return out
+
+
+def test_zoh_series_coefficients_in_arg_units():
+    """φ(x) = Σ x^k/(k+1)!, evaluated in arg = x log2(e): the coefficient of
+    arg^k is ln(2)^k/(k+1)!; the switch |x| < 0.1 is |arg| < 0.1 log2(e)."""
+    c = _consts("ssm_fwd_tma.cu", ["L1", "L2", "L3", "L4", "L5", "kSmall"])
+    for k in range(1, 6):
+        want = math.log(2.0) ** k / math.factorial(k + 1)
+        assert abs(c[f"L{k}"] - want) <= 2e-7 * want, (k, c[f"L{k}"], want)
+    assert abs(c["kSmall"] - 0.1 / math.log(2.0)) <= 1e-7
+
+
+def test_zoh_series_accuracy_over_its_range():
+    """With those coefficients the degree-5 series in arg stays within its
+    truncation error (x^6/7! < 3e-10 for |x| < 0.1) of φ over its range."""
+    c = _consts("ssm_fwd_tma.cu", ["L1", "L2", "L3", "L4", "L5", "kSmall"])
+    arg = np.linspace(-c["kSmall"], c["kSmall"], 2001)
+    x = arg * math.log(2.0)
+    exact = np.where(x == 0, 1.0, np.expm1(x) / np.where(x == 0, 1.0, x))
+    ser = 1 + arg * (c["L1"] + arg * (c["L2"] + arg * (c["L3"] + arg * (c["L4"] + arg * c["L5"]))))
+    assert np.max(np.abs(ser - exact) / exact) < 5e-9
