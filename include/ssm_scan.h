@@ -200,9 +200,10 @@ ssm_status_t ssm_selective_scan_bwd(const ssm_shape_t *shape,
  *  - Shapes whose scratch (ssm_selective_scan_bwd_scratch_bytes(shape, 0))
  *    exceeds SSM_NOALLOC_SCRATCH_BYTES are rejected with
  *    SSM_ERR_UNSUPPORTED before anything is launched.
- *  - The first call on a device looks up the array's device address (once
- *    per device, with that device current); make that first call before any
- *    stream capture.
+ *  - Every call looks up the array's device address on the current device
+ *    (a runtime query, no allocation); make the first call on a device
+ *    before any stream capture, since that first query also loads the
+ *    library's module on the device.
  *  - Every call on a device shares the one array and overwrites it: calls
  *    that overlap on the GPU (e.g. on two streams) race, so serialise them.
  *    Nothing of a previous call's contents is relied upon.

@@ -16,15 +16,13 @@ __device__ int g_ssm_device_error = 0;
 namespace ssm {
 
 int *device_error_word() {
-    static int *addr[64] = {nullptr};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    if (!addr[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_ssm_device_error) != cudaSuccess) return nullptr;
-        addr[dev] = static_cast<int *>(p);
-    }
-    return addr[dev];
+    // Looked up on every call (a cheap runtime query) rather than cached: no
+    // lock is needed between host threads, and an address from an earlier
+    // context of this device (after a cudaDeviceReset in the caller's
+    // process) is never reused.
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_ssm_device_error) != cudaSuccess) return nullptr;
+    return static_cast<int *>(p);
 }
 
 cudaError_t read_and_clear_device_error(int *value, cudaStream_t stream) {
@@ -200,6 +198,9 @@ ssm_status_t fwd_impl(const ssm_shape_t *shape, const ssm_options_t *opts, const
     p.vec_ok = ((size_t)shape->seqlen * es) % 16 == 0 && aligned16(u) && aligned16(delta) &&
                aligned16(B) && aligned16(C) && aligned16(out) && (!z || aligned16(z));
     cudaError_t e = ssm::launch_fwd(p, false, static_cast<cudaStream_t>(stream));
+    if (e == cudaErrorNotSupported && ssm::fwd_kernel_choice() == ssm::FwdKernel::kTma)
+        return fail(SSM_ERR_UNSUPPORTED,
+                    "SSM_FWD_KERNEL=tma: the TMA-fed forward does not cover this shape");
     if (e != cudaSuccess) return cuda_fail(e, "ssm_selective_scan_fwd launch");
     return ok();
 }

@@ -92,7 +92,7 @@ bool try_launch_fwd_tma(const FwdParams &p, cudaStream_t stream, cudaError_t *er
 ssm_status_t set_last_error(ssm_status_t status, const char *msg);
 
 // Device address of the error word that kernels set when a bounded wait
-// gives up (one word per device, looked up once per device); NULL on failure.
+// gives up (one word per device, looked up on every call); NULL on failure.
 int *device_error_word();
 // Copies the device error word to *value (after synchronising `stream`) and
 // clears it when set.

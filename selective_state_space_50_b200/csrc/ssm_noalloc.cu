@@ -10,8 +10,6 @@
 
 #include <stdio.h>
 
-#include <mutex>
-
 #include "ssm_internal.h"
 
 namespace {
@@ -22,25 +20,15 @@ constexpr size_t kScratchBytes = SSM_NOALLOC_SCRATCH_BYTES;
 // symbol, not a device address: kernels get the address looked up below.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_lookup_mutex;
-void *g_scratch_addr[kMaxDevices] = {nullptr};
-
-// Device address of g_noalloc_scratch on the current device, looked up once
-// per device (with that device current) and cached.
+// Device address of g_noalloc_scratch on the current device.  It is looked
+// up on every call (a cheap runtime query) rather than cached, so an address
+// from an earlier context of this device (after a cudaDeviceReset in the
+// caller's process) is never reused.
 cudaError_t scratch_address(void **out) {
-    int dev = -1;
-    cudaError_t e = cudaGetDevice(&dev);
+    void *p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_lookup_mutex);
-    if (!g_scratch_addr[dev]) {
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess) return e;
-        g_scratch_addr[dev] = p;
-    }
-    *out = g_scratch_addr[dev];
+    *out = p;
     return cudaSuccess;
 }
 

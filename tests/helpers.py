@@ -1,9 +1,19 @@
 """Shared helpers for the GPU tests: device copies of generated workloads and
 the tolerance checks used everywhere.
 
-Tolerances (fixed by the method's accuracy targets):
-  fp32 io:   |out - ref| <= 1e-4 * (1 + |ref|)  element-wise
-  bf16 io:   |out - ref| <= 2e-2 * (1 + |ref|)  element-wise
+Tolerances (fixed by the method's accuracy targets, tightened where the
+arithmetic allows):
+  fp32 io:   |out - ref| <= 1e-4 * (1 + |ref|)  element-wise, and
+             ||out - ref|| / ||ref|| <= 5e-5 normwise
+  bf16 io:   |out - ref| <= 1e-2 * (1 + |ref|)  element-wise, and
+             ||out - ref|| / ||ref|| <= 4e-3 normwise.
+             The stated bf16 target is 2e-2; the bound used is tighter.  A bf16
+             output is the kernel's fp32 value rounded to nearest: at most half
+             an ulp, 2^-8 |y| relative.  The SiLU gate on the hardware tanh adds
+             at most about 2^-11 |y|, and the fp32 scan itself far less, so
+             |out - ref| stays below 4.4e-3 |y| (the 1e-2 bound leaves 2x), and
+             rounding errors spread evenly over an ulp give a normwise error
+             near 2^-9 / sqrt(3) = 1.1e-3 (4e-3 leaves 3x).
   gradients: ||g - ref|| / ||ref|| <= 1e-3 per tensor, and element-wise
              |g - ref| <= 1e-2 * (|ref| + rms(ref))
 """
@@ -12,7 +22,8 @@ import torch
 
 from selective_state_space_50_b200.workloads import to_torch
 
-TOL = {"f32": 1e-4, "bf16": 2e-2}
+TOL = {"f32": 1e-4, "bf16": 1e-2}
+NORM_TOL = {"f32": 5e-5, "bf16": 4e-3}
 GRAD_NORM_TOL = 1e-3
 GRAD_ELEM_TOL = 1e-2
 
@@ -40,6 +51,8 @@ def to_f64(t: torch.Tensor) -> np.ndarray:
 
 
 def assert_close_io(got: np.ndarray, ref: np.ndarray, io_dtype: str, what: str = "out"):
+    """Element-wise and normwise check of a forward result against the fp64
+    oracle; prints both errors and returns the element-wise one."""
     tol = TOL[io_dtype]
     err = np.abs(got - ref)
     bound = tol * (1.0 + np.abs(ref))
@@ -48,7 +61,13 @@ def assert_close_io(got: np.ndarray, ref: np.ndarray, io_dtype: str, what: str =
         i = np.unravel_index(np.argmax(err / bound), err.shape)
         raise AssertionError(f"{what}: {bad.sum()} of {bad.size} outside {tol}*(1+|ref|); worst at "
                              f"{i}: got {got[i]!r} ref {ref[i]!r}")
-    return float((err / (1.0 + np.abs(ref))).max())
+    emax = float((err / (1.0 + np.abs(ref))).max()) if err.size else 0.0
+    nrm = float(np.linalg.norm(ref))
+    rel = float(np.linalg.norm(got - ref)) / nrm if nrm > 0 else float(np.linalg.norm(got))
+    print(f"{what}: max |e|/(1+|ref|) {emax:.3e}, normwise ||e||/||ref|| {rel:.3e}")
+    assert rel <= NORM_TOL[io_dtype], (f"{what}: normwise error {rel:.3e} above "
+                                      f"{NORM_TOL[io_dtype]:.0e}")
+    return emax
 
 
 def assert_close_grad(got: np.ndarray, ref: np.ndarray, what: str):

@@ -101,3 +101,34 @@ def test_zoh_step(N, io):
                                      c["C64"], c["D64"], c["z64"], c["bias64"], True, zoh=True)
     assert_close_io(out.double().cpu().numpy(), ref_out, io, "out")
     assert_close_io(c["state"].double().cpu().numpy(), ref_state, "f32", "state")
+
+
+@pytest.mark.parametrize("case", [
+    (2, 5, 70, 16, "f32", True, True, True, False, "neg_lognormal"),      # general forward
+    (2, 2400, 72, 16, "f32", True, True, True, False, "neg_lognormal"),   # TMA forward
+])
+def test_zoh_forward_at_series_switch(case):
+    """Δ·A straddles ±0.1, where the zero-order-hold factor switches from its
+    Taylor series to (Ā - 1)/(ΔA) (booiljung.github.io, "3.2 선택적 스캔
+    (Selective Scan) 알고리즘" §2.1: B̄ = (ΔA)⁻¹(exp(ΔA) - I)ΔB): A = -1 and
+    Δ in [0.05, 0.2] (softplus off, no bias), fp32 bound 1e-4 (1 + |y|)."""
+    w = small_workload(*case)
+    inp = generate(w, with_dout=True)
+    rng = np.random.default_rng(7)
+    A = np.full(inp["A"].shape, -1.0, dtype=np.float32)
+    dl = rng.uniform(0.05, 0.2, size=inp["delta"].shape).astype(np.float32)
+    bias = np.zeros(inp["delta_bias"].shape, dtype=np.float32)
+    for k, v in (("A", A), ("delta", dl), ("delta_bias", bias)):
+        inp[k], inp[k + "_f64"] = v, v.astype(np.float64)
+    x = dl.astype(np.float64) * -1.0
+    assert (x > -0.1).any() and (x < -0.1).any()
+    dv = to_device(inp, w)
+    out, last, _ = ssm_scan.selective_scan_fwd(dv["u"], dv["delta"], dv["A"], dv["B"], dv["C"],
+                                               dv["D"], dv["z"], dv["delta_bias"], False,
+                                               return_last_state=True, zoh=True)
+    torch.cuda.synchronize()
+    ref, rlast = oracle.fwd(inp["u_f64"], inp["delta_f64"], inp["A_f64"], inp["B_f64"],
+                            inp["C_f64"], inp["D_f64"], inp["z_f64"], inp["delta_bias_f64"],
+                            False, zoh=True)
+    assert_close_io(to_f64(out), ref, "f32")
+    assert_close_io(to_f64(last), rlast, "f32", "last_state")

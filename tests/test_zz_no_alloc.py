@@ -14,6 +14,7 @@ import ctypes
 import pytest
 import torch
 
+import oracle
 from selective_state_space_50_b200 import ssm_scan
 from selective_state_space_50_b200.workloads import Workload, generate, to_torch
 
@@ -32,6 +33,20 @@ def _cuda():
 GRADS = ("du", "ddelta", "dA", "dB", "dC", "dD", "dz", "ddelta_bias")
 
 
+_OUT = {}
+
+
+def _noalloc_into(dv, w):
+    """Calls the entry point on gradient buffers kept from the previous call,
+    so that the call itself is the only thing that could allocate."""
+    g = _OUT["g"]
+    shape = ssm_scan.make_shape(w.batch, w.dim, w.seqlen, w.dstate, dv["u"].dtype)
+    ssm_scan.bwd_noalloc_raw(shape, dv["u"], dv["delta"], dv["A"], dv["B"], dv["C"], dv["D"],
+                             dv["z"], dv["delta_bias"], w.softplus, dv["dout"], g["du"],
+                             g["ddelta"], g["dA"], g["dB"], g["dC"], g["dD"], g["dz"],
+                             g["ddelta_bias"])
+
+
 def _noalloc(dv, w, fill):
     shape = ssm_scan.make_shape(w.batch, w.dim, w.seqlen, w.dstate, dv["u"].dtype)
     f32 = dict(device="cuda", dtype=torch.float32)
@@ -46,6 +61,7 @@ def _noalloc(dv, w, fill):
                              g["ddelta"], g["dA"], g["dB"], g["dC"], g["dD"], g["dz"],
                              g["ddelta_bias"])
     torch.cuda.synchronize()
+    _OUT["g"] = g
     return g
 
 
@@ -53,16 +69,36 @@ def _noalloc(dv, w, fill):
 def test_noalloc_matches_regular_backward_on_two_calls(io):
     w = Workload("noalloc", 2, 300, 96, 16, io, seed=31, A_dist="neg_lognormal",
                  D_dist="u0.5_1.5")
-    dv = to_torch(generate(w, with_dout=True), w, "cuda")
+    inp = generate(w, with_dout=True)
+    dv = to_torch(inp, w, "cuda")
     ref = ssm_scan.selective_scan_bwd(dv["u"], dv["delta"], dv["A"], dv["B"], dv["C"], dv["D"],
                                       dv["z"], dv["delta_bias"], w.softplus, dv["dout"])
     torch.cuda.synchronize()
+    exact = oracle.bwd_workload(inp, w)
     # second call starts from the first call's scratch contents; outputs are
     # pre-filled with different junk each time
     for call, fill in enumerate((float("nan"), 1.0e30)):
         got = _noalloc(dv, w, fill)
         for k in GRADS:
             assert_close_grad(to_f64(got[k]), to_f64(ref[k]), f"call {call}: {k}")
+            assert_close_grad(to_f64(got[k]), exact[k], f"call {call}: {k} vs the fp64 oracle")
+
+
+def test_noalloc_allocates_no_device_memory():
+    """After a first call (which may load the library's module on the device),
+    further calls leave the device's free memory unchanged: the entry point
+    allocates nothing."""
+    w = Workload("noalloc", 2, 256, 160, 16, "bf16", seed=32, A_dist="neg_lognormal",
+                 D_dist="u0.5_1.5")
+    dv = to_torch(generate(w, with_dout=True), w, "cuda")
+    _noalloc(dv, w, 0.0)
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(3):
+        _noalloc_into(dv, w)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0, (free0, free1)
 
 
 def test_noalloc_rejects_shapes_beyond_its_buffer():
