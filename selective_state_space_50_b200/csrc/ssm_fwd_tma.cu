@@ -46,6 +46,9 @@
 #ifndef SSM_TMA_POLY_PAIRS
 #define SSM_TMA_POLY_PAIRS 0  // (state, step-pair) slots of 16 per block using ex2_poly2
 #endif
+#ifndef SSM_TMA_F32BC
+#define SSM_TMA_F32BC 1       // producer rewrites B/C as fp32 (32-step tiles)
+#endif
 #ifndef SSM_TMA_UNROLL
 #define SSM_TMA_UNROLL 2      // 8-step blocks unrolled in the recurrence loop
 #endif
@@ -89,14 +92,22 @@ struct TmaLayout {
     static constexpr int PIECE = 2 * N * PW;                   // one piece, two batch rows
     static constexpr int RAW_BC = NPIECE * PIECE;
     static constexpr int kBC0 = (3 * RAW_CH + 1023) / 1024 * 1024;
-    static constexpr int STAGE = (kBC0 + 2 * RAW_BC + 1023) / 1024 * 1024;
+    // With 32-step tiles the producer warp also rewrites each B and C tile as
+    // fp32 ([B or C][batch row][state][TT], 16-byte chunks swizzled so that
+    // the state groups of a warp read different banks): consumers then load
+    // four steps of B or C per 16-byte broadcast load, with no conversion.
+    static constexpr bool F32BC = SSM_TMA_F32BC && TT == 32;
+    static constexpr int BCF = 2 * 2 * N * TT;                 // floats of the fp32 copy
+    static constexpr int kBCF0 = align128(kBC0 + 2 * RAW_BC);
+    static constexpr int STAGE = (kBCF0 + (F32BC ? BCF * 4 : 0) + 1023) / 1024 * 1024;
     static constexpr int WS = TT + 4;                          // fp32 row stride (floats)
     static constexpr int WBUF = (2 + NT) * CPW * WS * 4;       // Δ, Δ·u, NT readout partials
     static constexpr int kW = STAGES * STAGE;
     static constexpr int kBar = kW + NWC * WBUF;
-    static constexpr int kTotal = kBar + 2 * STAGES * 8;
+    static constexpr int kTotal = kBar + 3 * STAGES * 8;
     static constexpr int kAlloc = kTotal + 1024;   // room to align the base to 1024 B
-    static constexpr int kThreads = (NWC + 1) * 32;
+    // consumer warps, the TMA warp and (with the fp32 B/C copy) a converter warp
+    static constexpr int kThreads = (NWC + 1 + (F32BC ? 1 : 0)) * 32;
     static constexpr int CHUNK = 8;                            // steps per prep/epilogue item
     static constexpr int ITEMS = CPW * (TT / CHUNK);           // (row, chunk) items per warp
     static_assert(kAlloc <= 227 * 1024, "shared memory budget");
@@ -182,7 +193,7 @@ __device__ __forceinline__ float rcp_approx(float x) {
 // write the per-row delta sums: the code is left out of the others, where
 // it measured 4 % slower even unused.
 template <typename T, int NT, int NS, int TT, int NWC, int STAGES, int FL>
-__global__ void __launch_bounds__((NWC + 1) * 32, 1)
+__global__ void __launch_bounds__(TmaLayout<T, NT, NS, TT, NWC, STAGES>::kThreads, 1)
 fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constant__ CUtensorMap m_u,
                const __grid_constant__ CUtensorMap m_z, const __grid_constant__ CUtensorMap m_B,
                const __grid_constant__ CUtensorMap m_C, const TmaFwdParams p) {
@@ -202,6 +213,7 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
     uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + Ly::kBar);
     uint64_t *empty = full + STAGES;
+    uint64_t *bcready = empty + STAGES;   // the producer wrote the fp32 B/C of a stage
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int G = gridDim.x;
@@ -216,6 +228,7 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(full + s, 1);
             mbar_init(empty + s, NWC);
+            mbar_init(bcready + s, 1);
         }
         fence_barrier_init();
     }
@@ -227,8 +240,16 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
         q1 = r0 + (int)((long long)(q + 1) * R / npass);
     };
 
+    // batch rows [b_lo, b_lo + nb) of the pass that tile kk belongs to
+    auto tile_batches = [&](int kk, int &b_lo, int &nb) {
+        int a0, a1;
+        pass_rows(kk / ntiles, a0, a1);
+        b_lo = a0 / p.dim;
+        nb = (a1 - 1) / p.dim - b_lo + 1;
+    };
+
     if (warp == NWC) {
-        // ------------------------------------------------------------ producer
+        // ------------------------------------------------------- TMA producer
         if (lane != 0) return;
         prefetch_tensormap(&m_delta);
         prefetch_tensormap(&m_u);
@@ -236,41 +257,82 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
         prefetch_tensormap(&m_B);
         prefetch_tensormap(&m_C);
         int issued = 0;
-        bool ok = true;
-        int s = 0, phase = 0, q = 0, tile = 0, q0 = 0, q1 = 0, b_lo = 0, nb = 1;
-        for (; issued < total && ok; ++issued) {
-            if (issued >= STAGES) {   // wait until every consumer left this stage
-                ok = mbar_wait_sleep(empty + s, phase ^ 1, p.err, 64);
-                if (!ok) break;
-            }
-            if (tile == 0) {
-                pass_rows(q, q0, q1);
-                b_lo = q0 / p.dim;
-                nb = (q1 - 1) / p.dim - b_lo + 1;
-            }
-            const int t0 = tile * TT;
-            uint8_t *st = smem + s * Ly::STAGE;
+        for (; issued < total; ++issued) {
+            const int si = issued % STAGES;
+            if (issued >= STAGES &&   // wait until every consumer left this stage
+                !mbar_wait_sleep(empty + si, ((issued / STAGES) & 1) ^ 1, p.err, 64))
+                break;
+            int a0, a1, b_lo, nb;
+            pass_rows(issued / ntiles, a0, a1);
+            tile_batches(issued, b_lo, nb);
+            const int t0 = (issued % ntiles) * TT;
+            uint8_t *st = smem + si * Ly::STAGE;
             const uint32_t bytes = (uint32_t)(p.rows_max * Ly::RAW_ROW * (has_z ? 3 : 2) +
                                               2 * nb * N * Ly::RAW_ROW);
-            mbar_arrive_expect_tx(full + s, bytes);
-            tma_load_2d(st, &m_delta, t0, q0, full + s);
-            tma_load_2d(st + Ly::RAW_CH, &m_u, t0, q0, full + s);
-            if (has_z) tma_load_2d(st + 2 * Ly::RAW_CH, &m_z, t0, q0, full + s);
+            mbar_arrive_expect_tx(full + si, bytes);
+            tma_load_2d(st, &m_delta, t0, a0, full + si);
+            tma_load_2d(st + Ly::RAW_CH, &m_u, t0, a0, full + si);
+            if (has_z) tma_load_2d(st + 2 * Ly::RAW_CH, &m_z, t0, a0, full + si);
             for (int bs = 0; bs < nb; ++bs)
                 for (int pc = 0; pc < Ly::NPIECE; ++pc) {
                     const int off = Ly::kBC0 + pc * Ly::PIECE + bs * N * Ly::PW;
                     const int x = t0 + pc * (Ly::PW / (int)sizeof(T));
-                    tma_load_2d(st + off, &m_B, x, (b_lo + bs) * N, full + s);
-                    tma_load_2d(st + off + Ly::RAW_BC, &m_C, x, (b_lo + bs) * N, full + s);
+                    tma_load_2d(st + off, &m_B, x, (b_lo + bs) * N, full + si);
+                    tma_load_2d(st + off + Ly::RAW_BC, &m_C, x, (b_lo + bs) * N, full + si);
                 }
-            if (++s == STAGES) { s = 0; phase ^= 1; }
-            if (++tile == ntiles) { tile = 0; ++q; }
         }
         // Never leave while a copy may still write shared memory: the last
         // STAGES loads are the only ones no consumer is known to have seen.
-        for (int kg = (issued > STAGES ? issued - STAGES : 0); kg < issued; ++kg)
-            if (!mbar_wait(full + (kg % STAGES), (kg / STAGES) & 1, p.err)) break;
+        for (int kk = (issued > STAGES ? issued - STAGES : 0); kk < issued; ++kk)
+            if (!mbar_wait(full + (kk % STAGES), (kk / STAGES) & 1, p.err)) break;
         return;
+    }
+    if constexpr (Ly::F32BC) {
+        if (warp == NWC + 1) {
+            // ------------------------------------------------ B/C converter
+            // Each tile's B and C, once landed, rewritten as fp32 rows in the
+            // stage's fp32 area (16-byte chunks swizzled by row / NS), then
+            // announced on bcready.  The stage was refilled only after every
+            // consumer left it, so its fp32 area is free.
+            constexpr int CH = TT / 4;                 // fp32 16-byte chunks per row
+            constexpr int PER_LANE = N * CH / 32;      // (state, chunk) items per lane
+            static_assert(N * CH % 32 == 0, "items per lane");
+            for (int kk = 0; kk < total; ++kk) {
+                const int si = kk % STAGES;
+                if (!__all_sync(0xffffffffu, mbar_wait(full + si, (kk / STAGES) & 1, p.err))) return;
+                int b_lo, nb;
+                tile_batches(kk, b_lo, nb);
+                const uint8_t *raw = smem + si * Ly::STAGE + Ly::kBC0;
+                float *dst = reinterpret_cast<float *>(smem + si * Ly::STAGE + Ly::kBCF0);
+                for (int which = 0; which < 2; ++which)
+                    for (int bs = 0; bs < nb; ++bs) {
+#pragma unroll
+                        for (int r = 0; r < PER_LANE; ++r) {
+                            const int it = lane + 32 * r;
+                            const int ch = it % CH, rr = bs * N + it / CH;
+                            constexpr int ES = (int)sizeof(T);
+                            const int byte = ch * 4 * ES;
+                            const int pc = byte / Ly::PW, in = byte % Ly::PW;
+                            int rch = in >> 4;
+                            if constexpr (Ly::SWZ) rch ^= (rr & 7);
+                            const uint8_t *src = raw + which * Ly::RAW_BC + pc * Ly::PIECE + rr * Ly::PW + rch * 16;
+                            float4 v;
+                            if constexpr (ES == 2) {
+                                const uint2 q2 = *reinterpret_cast<const uint2 *>(src + (in & 15));
+                                v = make_float4(__uint_as_float(q2.x << 16), __uint_as_float(q2.x & 0xffff0000u),
+                                                __uint_as_float(q2.y << 16), __uint_as_float(q2.y & 0xffff0000u));
+                            } else {
+                                v = *reinterpret_cast<const float4 *>(src);
+                            }
+                            float *drow = dst + (which * 2 * N + rr) * TT;
+                            *reinterpret_cast<float4 *>(drow + ((ch ^ ((rr / NS) & 7)) << 2)) = v;
+                        }
+                    }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bcready + si);
+            }
+            return;
+        }
     }
 
     // ---------------------------------------------------------------- consumers
@@ -338,7 +400,11 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
             }
         }
         // every lane waits; the warp leaves together if any wait gave up
-        if (!__all_sync(0xffffffffu, mbar_wait(full + s, phase, p.err))) return;
+        {
+            bool ok = mbar_wait(full + s, phase, p.err);
+            if constexpr (Ly::F32BC) ok = ok && mbar_wait(bcready + s, phase, p.err);
+            if (!__all_sync(0xffffffffu, ok)) return;
+        }
 
         if (wrow0 < wend) {
             const uint8_t *st = smem + s * Ly::STAGE;
@@ -373,7 +439,6 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                         du[v0 + k] = u2.x; du[v0 + k + 1] = u2.y;
                     }
                 }
-#pragma unroll
                 if (kDsum && p.delta_sum) {
 #pragma unroll
                     for (int k = 0; k < CHUNK; ++k) dsum[i] += dt[k];
@@ -400,6 +465,11 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                 return reinterpret_cast<const T *>(base + pc * Ly::PIECE + rr * Ly::PW + (chunk << 4));
             };
             const int rr0 = bsel * N + g * NS;
+            // fp32 copy of B and C: rows of this lane's states, and the chunk
+            // swizzle key of those rows (one per lane)
+            const float *bcfB = reinterpret_cast<const float *>(st + Ly::kBCF0) + rr0 * TT;
+            const float *bcfC = bcfB + 2 * N * TT;
+            const int bkey = (rr0 / NS) & 7;
             float *myY = wY + (g * CPW + c) * WS;
             float *ck_row = (live && ckpt) ? ckpt + (size_t)(wrow0 + c) * p.n_ckpt * N + g * NS : nullptr;
             static_assert(SSM_CKPT_CHUNK == 8, "checkpoints are written per 8-step block");
@@ -432,8 +502,20 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
 #pragma unroll
                     for (int j = 0; j < NS; ++j) {
                         float2 bq[4], cq[4];
-                        load_pairs8_at<T>(bc_chunk(rawB, rr0 + j, tb), bc_chunk(rawB, rr0 + j, tb + 4), bq);
-                        load_pairs8_at<T>(bc_chunk(rawC, rr0 + j, tb), bc_chunk(rawC, rr0 + j, tb + 4), cq);
+                        if constexpr (Ly::F32BC) {
+                            const int c0 = ((tb >> 2) ^ bkey) << 2, c1 = (((tb >> 2) + 1) ^ bkey) << 2;
+                            const float4 b0 = *reinterpret_cast<const float4 *>(bcfB + j * TT + c0);
+                            const float4 b1 = *reinterpret_cast<const float4 *>(bcfB + j * TT + c1);
+                            const float4 e0 = *reinterpret_cast<const float4 *>(bcfC + j * TT + c0);
+                            const float4 e1 = *reinterpret_cast<const float4 *>(bcfC + j * TT + c1);
+                            bq[0] = make_float2(b0.x, b0.y); bq[1] = make_float2(b0.z, b0.w);
+                            bq[2] = make_float2(b1.x, b1.y); bq[3] = make_float2(b1.z, b1.w);
+                            cq[0] = make_float2(e0.x, e0.y); cq[1] = make_float2(e0.z, e0.w);
+                            cq[2] = make_float2(e1.x, e1.y); cq[3] = make_float2(e1.z, e1.w);
+                        } else {
+                            load_pairs8_at<T>(bc_chunk(rawB, rr0 + j, tb), bc_chunk(rawB, rr0 + j, tb + 4), bq);
+                            load_pairs8_at<T>(bc_chunk(rawC, rr0 + j, tb), bc_chunk(rawC, rr0 + j, tb + 4), cq);
+                        }
 #pragma unroll
                         for (int pp = 0; pp < 4; ++pp) {
                             const float2 arg = __fmul2_rn(dtp[pp], A2d[j]);
@@ -588,7 +670,10 @@ SSM_TMA_CFG(bf16_t, 16, 2, 9, SSM_TMA_STAGES)
 #ifndef SSM_TMA_NWC_BF16_N16
 #define SSM_TMA_NWC_BF16_N16 12
 #endif
-SSM_TMA_CFG(bf16_t, 16, 4, SSM_TMA_NWC_BF16_N16, SSM_TMA_STAGES)
+#ifndef SSM_TMA_STAGES_NT4
+#define SSM_TMA_STAGES_NT4 SSM_TMA_STAGES
+#endif
+SSM_TMA_CFG(bf16_t, 16, 4, SSM_TMA_NWC_BF16_N16, SSM_TMA_STAGES_NT4)
 SSM_TMA_CFG(bf16_t, 16, 8, 12, 3)
 SSM_TMA_CFG(bf16_t, 16, 16, 7, 3)
 SSM_TMA_CFG(bf16_t, 32, 4, 12, SSM_TMA_STAGES)
