@@ -49,6 +49,12 @@
 #ifndef SSM_TMA_F32BC
 #define SSM_TMA_F32BC 1       // producer rewrites B/C as fp32 (32-step tiles)
 #endif
+#ifndef SSM_TMA_WAIT_SUSPEND
+#define SSM_TMA_WAIT_SUSPEND 0    // waits suspend in the barrier unit instead of polling
+#endif
+#ifndef SSM_TMA_STEP_MAJOR
+#define SSM_TMA_STEP_MAJOR 1      // recurrence loop ordered step-major (fp32 B/C, Δ·B only)
+#endif
 #ifndef SSM_TMA_UNROLL
 #define SSM_TMA_UNROLL 2      // 8-step blocks unrolled in the recurrence loop
 #endif
@@ -59,6 +65,7 @@ namespace {
 
 constexpr int kTmaUnroll = SSM_TMA_UNROLL;
 constexpr int kPolyPairs = SSM_TMA_POLY_PAIRS;
+constexpr bool kStepMajor = SSM_TMA_STEP_MAJOR != 0;
 
 constexpr int align128(int x) { return (x + 127) / 128 * 128; }
 
@@ -299,7 +306,11 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
             static_assert(N * CH % 32 == 0, "items per lane");
             for (int kk = 0; kk < total; ++kk) {
                 const int si = kk % STAGES;
+#if SSM_TMA_WAIT_SUSPEND
+                if (!__all_sync(0xffffffffu, mbar_wait_suspend(full + si, (kk / STAGES) & 1, p.err))) return;
+#else
                 if (!__all_sync(0xffffffffu, mbar_wait(full + si, (kk / STAGES) & 1, p.err))) return;
+#endif
                 int b_lo, nb;
                 tile_batches(kk, b_lo, nb);
                 const uint8_t *raw = smem + si * Ly::STAGE + Ly::kBC0;
@@ -401,8 +412,13 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
         }
         // every lane waits; the warp leaves together if any wait gave up
         {
+#if SSM_TMA_WAIT_SUSPEND
+            bool ok = mbar_wait_suspend(full + s, phase, p.err);
+            if constexpr (Ly::F32BC) ok = ok && mbar_wait_suspend(bcready + s, phase, p.err);
+#else
             bool ok = mbar_wait(full + s, phase, p.err);
             if constexpr (Ly::F32BC) ok = ok && mbar_wait(bcready + s, phase, p.err);
+#endif
             if (!__all_sync(0xffffffffu, ok)) return;
         }
 
@@ -499,6 +515,45 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                     float2 y2[4];
 #pragma unroll
                     for (int pp = 0; pp < 4; ++pp) y2[pp] = make_float2(0.f, 0.f);
+                    if constexpr (Ly::F32BC && !ZOH && !kPoly && kStepMajor) {
+                        // step-major order: per pair of steps, every state's
+                        // exponentials, then the NS independent recurrence
+                        // chains side by side, then the readout
+#pragma unroll
+                        for (int hb = 0; hb < 2; ++hb) {
+                            const int cc = (((tb >> 2) + hb) ^ bkey) << 2;
+                            float4 Bv[NS], Cv[NS];
+#pragma unroll
+                            for (int j = 0; j < NS; ++j) {
+                                Bv[j] = *reinterpret_cast<const float4 *>(bcfB + j * TT + cc);
+                                Cv[j] = *reinterpret_cast<const float4 *>(bcfC + j * TT + cc);
+                            }
+#pragma unroll
+                            for (int pq = 0; pq < 2; ++pq) {
+                                const int pp = 2 * hb + pq;
+                                float2 a[NS], beta[NS];
+                                float hA[NS];
+#pragma unroll
+                                for (int j = 0; j < NS; ++j) {
+                                    const float2 arg = __fmul2_rn(dtp[pp], A2d[j]);
+                                    a[j] = make_float2(ex2(arg.x), ex2(arg.y));
+                                    const float2 bb = pq ? make_float2(Bv[j].z, Bv[j].w) : make_float2(Bv[j].x, Bv[j].y);
+                                    beta[j] = __fmul2_rn(dup[pp], bb);
+                                }
+#pragma unroll
+                                for (int j = 0; j < NS; ++j) hA[j] = fmaf(a[j].x, h[j], beta[j].x);
+#pragma unroll
+                                for (int j = 0; j < NS; ++j) h[j] = fmaf(a[j].y, hA[j], beta[j].y);
+                                float2 yy = make_float2(0.f, 0.f);
+#pragma unroll
+                                for (int j = 0; j < NS; ++j) {
+                                    const float2 cv = pq ? make_float2(Cv[j].z, Cv[j].w) : make_float2(Cv[j].x, Cv[j].y);
+                                    yy = __ffma2_rn(cv, make_float2(hA[j], h[j]), yy);
+                                }
+                                y2[pp] = yy;
+                            }
+                        }
+                    } else {
 #pragma unroll
                     for (int j = 0; j < NS; ++j) {
                         float2 bq[4], cq[4];
@@ -532,6 +587,7 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                             h[j] = h1;
                             y2[pp] = __ffma2_rn(cq[pp], make_float2(h0, h1), y2[pp]);
                         }
+                    }
                     }
                     *reinterpret_cast<float4 *>(myY + tb) = make_float4(y2[0].x, y2[0].y, y2[1].x, y2[1].y);
                     *reinterpret_cast<float4 *>(myY + tb + 4) = make_float4(y2[2].x, y2[2].y, y2[3].x, y2[3].y);

@@ -53,6 +53,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+// As mbar_try_wait, with a suspend-time hint: a thread whose phase is not yet
+// complete may be suspended (not polling) for up to `ns` nanoseconds, and
+// resumes when the phase completes.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t *bar, uint32_t parity, uint32_t ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Non-blocking test of the phase with the given parity (acquire on success).
 __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
@@ -75,6 +90,22 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *e
     const long long t0 = clock64();
     while (!mbar_try_wait(bar, parity)) {
         if (clock64() - t0 > budget) {
+            atomicExch(err, kErrWaitTimeout);
+            return false;
+        }
+    }
+    return true;
+}
+
+// As mbar_wait, but the waiting thread is suspended by the barrier unit
+// between checks (suspend-time hint of about 0.1 ms per check) instead of
+// spinning, so a warp that waits takes no issue slots from the warps that
+// work on the same SM sub-partition.
+__device__ __forceinline__ bool mbar_wait_suspend(uint64_t *bar, uint32_t parity, int *err) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait_hint(bar, parity, 100000u)) {
+        if (clock64() - t0 > kWaitBudgetCycles) {
             atomicExch(err, kErrWaitTimeout);
             return false;
         }
