@@ -289,6 +289,7 @@ def run_ours(args, world, rank, local):
     last = torch.empty(w.batch, w.dim, w.dstate, device=dev, dtype=torch.float32)
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    nws = 0   # workspace of the two-level scan (forward workloads only)
     if fwdbwd:
         ck = torch.empty(ssm_scan.ckpt_numel(shape), device=dev, dtype=torch.float32)
         f32 = dict(device=dev, dtype=torch.float32)
@@ -369,9 +370,15 @@ def run_ours(args, world, rank, local):
             ssm_scan.fwd_raw(shape, dv["u"], dv["delta"], dv["A"], dv["B"], dv["C"], dv["D"],
                              dv["z"], dv["delta_bias"], True, out, last, None, stream)
     else:
+        # shapes with long sequences over few channel rows take the two-level
+        # scan along the sequence (three launches), with its workspace
+        nws = ssm_scan.fwd_workspace_bytes(shape, True, args.zoh)
+        ws = torch.empty(nws // 4, device=dev, dtype=torch.float32) if nws else None
+
         def fwd():
             ssm_scan.fwd_raw(shape, dv["u"], dv["delta"], dv["A"], dv["B"], dv["C"], dv["D"],
-                             dv["z"], dv["delta_bias"], True, out, last, None, stream, zoh=args.zoh)
+                             dv["z"], dv["delta_bias"], True, out, last, None, stream, zoh=args.zoh,
+                             workspace=ws)
 
     for _ in range(max(3, args.warmup)):
         flush.zero_()
@@ -475,6 +482,7 @@ def run_ours(args, world, rank, local):
 
     if rank != 0:
         return
+    chunked = not (fwdbwd or proj or args.segments > 1) and nws > 0
     peaks, peak_src = measured_peaks()
     mean_s = t_dev / args.steps
     # one exponential per (step, state) in the forward, and one more in the
@@ -517,10 +525,14 @@ def run_ours(args, world, rank, local):
         # segments: S pass-1 scans (the TMA forward also sums Δ), the combine,
         # S - 1 pass-2 scans
         "gpu_launches": args.steps * (3 if proj else 2 if fwdbwd else
-                                      (2 * args.segments if args.segments > 1 else 1)),
+                                      (2 * args.segments if args.segments > 1 else
+                                       3 if chunked else 1)),
     }
     if args.zoh:
         line["config"]["discretization"] = "zero-order hold"
+    if chunked:
+        line["config"]["step"] = ("two-level scan along the sequence: chunk summaries, carry "
+                                  "combine, every chunk from its carry-in (3 launches)")
     if seg_info:
         line["segments"] = seg_info
         line["config"]["step"] = (f"sequence cut into {args.segments} segments: pass 1 over all, "

@@ -147,6 +147,42 @@ ssm_status_t ssm_selective_scan_fwd_ex(const ssm_shape_t *shape, const ssm_optio
                                        void *stream);
 
 /*
+ * Workspace for the two-level scan along the sequence (booiljung.github.io,
+ * "3.2 선택적 스캔(Selective Scan) 알고리즘" §2.2: chunk summaries (Ā product,
+ * local state) composed with the associative operator (a_j, b_j)•(a_i, b_i) =
+ * (a_j a_i, a_j b_i + b_j)).  When a shape has long sequences over few
+ * channel rows (fewer than 64 rows per SM), ssm_selective_scan_fwd_ws cuts
+ * the sequence into K chunks of whole 128-step blocks and runs three launches
+ * on `stream`: the summaries of chunks 0..K-2 (end state from a zero state,
+ * and Σ_t Δ_t), the exclusive combine of the summaries (the state entering
+ * each chunk), and every chunk from its entering state.
+ *
+ * ssm_selective_scan_fwd_workspace_bytes: the bytes of workspace that
+ *   ssm_selective_scan_fwd_ws uses for this shape on the current device (0:
+ *   the one-pass forward is used, and the workspace may be NULL).  The plan
+ *   assumes 16-byte aligned rows; with unaligned pointers the one-pass path
+ *   runs and the workspace is not touched.
+ * ssm_selective_scan_fwd_ws: ssm_selective_scan_fwd_ex with a caller-owned
+ *   device workspace (16-byte aligned, `workspace_bytes` long; its contents
+ *   on entry are ignored and on return undefined).  Results match the
+ *   one-pass forward to within fp32 rounding (the chunks' states are joined
+ *   in fp32).  Calls that share a workspace must not overlap on the GPU.
+ * Errors: as ssm_selective_scan_fwd_ex, plus SSM_ERR_INVALID_ARG when the
+ * workspace is smaller than the plan needs.
+ */
+ssm_status_t ssm_selective_scan_fwd_workspace_bytes(const ssm_shape_t *shape,
+                                                    const ssm_options_t *opts, size_t *bytes);
+
+ssm_status_t ssm_selective_scan_fwd_ws(const ssm_shape_t *shape, const ssm_options_t *opts,
+                                       const void *u, const void *delta,
+                                       const float *A, const void *B, const void *C,
+                                       const float *D, const void *z,
+                                       const float *delta_bias,
+                                       void *out, float *last_state, float *ckpt,
+                                       void *workspace, size_t workspace_bytes,
+                                       void *stream);
+
+/*
  * Bytes of device scratch that ssm_selective_scan_bwd needs: 0 when the
  * caller passes the forward's checkpoints (have_ckpt != 0), otherwise the
  * size of a checkpoint buffer, which the backward fills itself first.

@@ -164,7 +164,8 @@ namespace {
 ssm_status_t fwd_impl(const ssm_shape_t *shape, const ssm_options_t *opts, const void *u,
                       const void *delta, const float *A, const void *B, const void *C,
                       const float *D, const void *z, const float *delta_bias, const float *h0,
-                      void *out, float *last_state, float *ckpt, float *delta_sum, void *stream) {
+                      void *out, float *last_state, float *ckpt, float *delta_sum, void *workspace,
+                      size_t workspace_bytes, void *stream) {
     SSM_TRY(check_shape(shape));
     SSM_TRY(check_options(opts));
     const size_t es = esize(shape->io_dtype);
@@ -197,7 +198,17 @@ ssm_status_t fwd_impl(const ssm_shape_t *shape, const ssm_options_t *opts, const
     p.io_bf16 = shape->io_dtype == SSM_BF16;
     p.vec_ok = ((size_t)shape->seqlen * es) % 16 == 0 && aligned16(u) && aligned16(delta) &&
                aligned16(B) && aligned16(C) && aligned16(out) && (!z || aligned16(z));
-    cudaError_t e = ssm::launch_fwd(p, false, static_cast<cudaStream_t>(stream));
+    cudaError_t e;
+    const size_t need = workspace ? ssm::fwd_chunk_plan(p, nullptr, nullptr) : 0;
+    if (need > 0 && ssm::fwd_kernel_choice() == ssm::FwdKernel::kAuto) {
+        if (workspace_bytes < need)
+            return fail(SSM_ERR_INVALID_ARG, "workspace_bytes %zu < %zu needed for this shape",
+                        workspace_bytes, need);
+        SSM_TRY(check_ptr(workspace, "workspace", 16, true));
+        e = ssm::launch_fwd_chunked(p, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+    } else {
+        e = ssm::launch_fwd(p, false, static_cast<cudaStream_t>(stream));
+    }
     if (e == cudaErrorNotSupported && ssm::fwd_kernel_choice() == ssm::FwdKernel::kTma)
         return fail(SSM_ERR_UNSUPPORTED,
                     "SSM_FWD_KERNEL=tma: the TMA-fed forward does not cover this shape");
@@ -215,7 +226,31 @@ ssm_status_t ssm_selective_scan_fwd_ex(const ssm_shape_t *shape, const ssm_optio
                                        const float *delta_bias, void *out, float *last_state,
                                        float *ckpt, void *stream) {
     return fwd_impl(shape, opts, u, delta, A, B, C, D, z, delta_bias, nullptr, out, last_state, ckpt,
-                    nullptr, stream);
+                    nullptr, nullptr, 0, stream);
+}
+
+ssm_status_t ssm_selective_scan_fwd_workspace_bytes(const ssm_shape_t *shape,
+                                                    const ssm_options_t *opts, size_t *bytes) {
+    SSM_TRY(check_shape(shape));
+    SSM_TRY(check_options(opts));
+    if (!bytes) return fail(SSM_ERR_INVALID_ARG, "bytes is NULL");
+    ssm::FwdParams p{};
+    p.batch = shape->batch; p.dim = shape->dim; p.L = shape->seqlen; p.N = shape->dstate;
+    p.zoh = opts->discretization == SSM_DISC_ZOH;
+    p.io_bf16 = shape->io_dtype == SSM_BF16;
+    p.vec_ok = ((size_t)shape->seqlen * esize(shape->io_dtype)) % 16 == 0;
+    *bytes = ssm::fwd_chunk_plan(p, nullptr, nullptr);
+    return ok();
+}
+
+ssm_status_t ssm_selective_scan_fwd_ws(const ssm_shape_t *shape, const ssm_options_t *opts,
+                                       const void *u, const void *delta, const float *A,
+                                       const void *B, const void *C, const float *D, const void *z,
+                                       const float *delta_bias, void *out, float *last_state,
+                                       float *ckpt, void *workspace, size_t workspace_bytes,
+                                       void *stream) {
+    return fwd_impl(shape, opts, u, delta, A, B, C, D, z, delta_bias, nullptr, out, last_state, ckpt,
+                    nullptr, workspace, workspace_bytes, stream);
 }
 
 ssm_status_t ssm_selective_scan_fwd_segment(const ssm_shape_t *shape, const ssm_options_t *opts,
@@ -225,7 +260,7 @@ ssm_status_t ssm_selective_scan_fwd_segment(const ssm_shape_t *shape, const ssm_
                                             void *out, float *last_state, float *ckpt,
                                             float *delta_sum, void *stream) {
     return fwd_impl(shape, opts, u, delta, A, B, C, D, z, delta_bias, h0, out, last_state, ckpt,
-                    delta_sum, stream);
+                    delta_sum, nullptr, 0, stream);
 }
 
 ssm_status_t ssm_scan_combine_carries(int nseg, int batch, int dim, int dstate, const float *A,

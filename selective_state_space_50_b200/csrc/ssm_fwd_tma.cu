@@ -55,6 +55,9 @@
 #ifndef SSM_TMA_STEP_MAJOR
 #define SSM_TMA_STEP_MAJOR 1      // recurrence loop ordered step-major (fp32 B/C, Δ·B only)
 #endif
+#ifndef SSM_TMA_SUM_POLY
+#define SSM_TMA_SUM_POLY 1        // quarters of a lane's states with FMA-pipe exponentials in chunk summaries
+#endif
 #ifndef SSM_TMA_UNROLL
 #define SSM_TMA_UNROLL 2      // 8-step blocks unrolled in the recurrence loop
 #endif
@@ -66,6 +69,7 @@ namespace {
 constexpr int kTmaUnroll = SSM_TMA_UNROLL;
 constexpr int kPolyPairs = SSM_TMA_POLY_PAIRS;
 constexpr bool kStepMajor = SSM_TMA_STEP_MAJOR != 0;
+constexpr int kSumPolyStates = SSM_TMA_SUM_POLY;
 
 constexpr int align128(int x) { return (x + 127) / 128 * 128; }
 
@@ -77,6 +81,15 @@ struct TmaFwdParams {
     float *last_state, *ckpt;
     int P;          // batch * dim channel rows
     int dim, L, n_ckpt;
+    // Time chunks (the two-level scan along L): the launch covers chunks
+    // 0..K-1 of Lc steps each (the last one ends at L); the CTAs are split
+    // evenly over the chunks, and a CTA's rows all lie in its chunk.  With
+    // K = 1 (Lc = L) the launch is one ordinary pass over the sequence.
+    // Chunk k's copy of row r is the virtual row v = k P + r; `virt` says
+    // bit 1: h0 is indexed by virtual row; bit 2: last_state and delta_sum
+    // are indexed by virtual row (else by row, and last_state is written by
+    // the last chunk only).
+    int K, Lc, virt;
     int softplus, has_z;
     int rows_max;   // rows of one pass (= box height of the per-channel maps)
     int *err;       // device error word
@@ -196,9 +209,11 @@ __device__ __forceinline__ float rcp_approx(float x) {
 // FL >= 0: the gate, softplus and checkpoint options are compile-time bits
 // (1: gate z, 2: softplus, 4: checkpoints); B̄ = Δ B.  FL = -1: the options
 // are read at run time; B̄ = Δ B.  FL = -2: options at run time, zero-order
-// hold B̄ = φ(Δ A) Δ B.  Only the run-time-option kernels (FL < 0) can also
-// write the per-row delta sums: the code is left out of the others, where
-// it measured 4 % slower even unused.
+// hold B̄ = φ(Δ A) Δ B.  FL = -3 / -4: chunk summaries of the two-level scan
+// (no readout, no output), with / without softplus: each row's end state
+// from a zero state, and Σ Δ.  Only the run-time-option kernels (FL < 0) can also write the per-row
+// delta sums: the code is left out of the others, where it measured 4 %
+// slower even unused.
 template <typename T, int NT, int NS, int TT, int NWC, int STAGES, int FL>
 __global__ void __launch_bounds__(TmaLayout<T, NT, NS, TT, NWC, STAGES>::kThreads, 1)
 fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constant__ CUtensorMap m_u,
@@ -209,10 +224,11 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
     constexpr int IPL = Ly::ITEMS / 32;   // prep/epilogue items per lane
     constexpr int CPR = TT / CHUNK;       // chunks per row
     constexpr bool ZOH = FL == -2;
+    constexpr bool kSummary = FL == -3 || FL == -4;
     constexpr bool kDsum = FL < 0;   // delta sums only in the run-time-option kernels
-    const bool has_z = FL < 0 ? p.has_z != 0 : (FL & 1) != 0;
-    const bool softplus = FL < 0 ? p.softplus != 0 : (FL & 2) != 0;
-    float *const ckpt = (FL < 0 || (FL & 4)) ? p.ckpt : nullptr;
+    const bool has_z = kSummary ? false : FL < 0 ? p.has_z != 0 : (FL & 1) != 0;
+    const bool softplus = kSummary ? FL == -3 : FL < 0 ? p.softplus != 0 : (FL & 2) != 0;
+    float *const ckpt = kSummary ? nullptr : (FL < 0 || (FL & 4)) ? p.ckpt : nullptr;
 
     extern __shared__ __align__(128) uint8_t smem_raw[];
     // 1024-byte aligned base: the 128B-swizzle pattern of the B/C tiles repeats
@@ -223,12 +239,19 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
     uint64_t *bcready = empty + STAGES;   // the producer wrote the fp32 B/C of a stage
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    // this CTA's time chunk kc (CTAs [g0, g1) share it) and its rows [r0, r1)
     const int G = gridDim.x;
-    const int r0 = (int)((long long)blockIdx.x * p.P / G);
-    const int r1 = (int)((long long)(blockIdx.x + 1) * p.P / G);
+    const int kc = (int)((long long)blockIdx.x * p.K / G);
+    const int g0 = (int)(((long long)kc * G + p.K - 1) / p.K);
+    const int g1 = (int)(((long long)(kc + 1) * G + p.K - 1) / p.K);
+    const int r0 = (int)((long long)(blockIdx.x - g0) * p.P / (g1 - g0));
+    const int r1 = (int)((long long)(blockIdx.x - g0 + 1) * p.P / (g1 - g0));
     const int R = r1 - r0;
+    const int T0 = kc * p.Lc;                     // the chunk's steps [T0, T1)
+    const int T1 = min(p.L, T0 + p.Lc);
+    const long long voff = (long long)kc * p.P;   // virtual row of row 0
     const int npass = (R + p.rows_max - 1) / p.rows_max;
-    const int ntiles = (p.L + TT - 1) / TT;
+    const int ntiles = (T1 - T0 + TT - 1) / TT;
     const int total = npass * ntiles;
 
     if (threadIdx.x == 0) {
@@ -272,7 +295,7 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
             int a0, a1, b_lo, nb;
             pass_rows(issued / ntiles, a0, a1);
             tile_batches(issued, b_lo, nb);
-            const int t0 = (issued % ntiles) * TT;
+            const int t0 = T0 + (issued % ntiles) * TT;
             uint8_t *st = smem + si * Ly::STAGE;
             const uint32_t bytes = (uint32_t)(p.rows_max * Ly::RAW_ROW * (has_z ? 3 : 2) +
                                               2 * nb * N * Ly::RAW_ROW);
@@ -377,7 +400,7 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
         if (tile == 0) {
             pass_rows(q, q0, q1);
         }
-        const int t0 = tile * TT;
+        const int t0 = T0 + tile * TT;
         const int wrow0 = q0 + warp * rpw;   // first row of this warp in the pass
         const int wend = min(wrow0 + rpw, q1);
         if (tile == 0) {
@@ -395,7 +418,7 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                     const float ia = 1.f / av;
                     iAd[j] = make_float2(ia, ia);
                 }
-                h[j] = (live && p.h0) ? p.h0[(size_t)row * N + g * NS + j] : 0.f;
+                h[j] = (live && p.h0) ? p.h0[(size_t)((p.virt & 1) ? voff + row : row) * N + g * NS + j] : 0.f;
                 neg = neg && a <= 0.f;
             }
             poly_ok = __all_sync(0xffffffffu, neg);
@@ -428,7 +451,7 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
             const T *rawU = reinterpret_cast<const T *>(st + Ly::RAW_CH) + warp * rpw * TT;
             const T *rawZ = reinterpret_cast<const T *>(st + 2 * Ly::RAW_CH) + warp * rpw * TT;
             // (1) Δ and Δ·u, once per element (pairs of steps in f32x2 math)
-            const bool full_tile = t0 + TT <= p.L;
+            const bool full_tile = t0 + TT <= T1;
 #pragma unroll
             for (int i = 0; i < IPL; ++i) {
                 const int it = lane + 32 * i, rl = it / CPR, t = (it % CPR) * CHUNK;
@@ -444,8 +467,8 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                         const float2 r = __fadd2_rn(make_float2(dr[k], dr[k + 1]), make_float2(bias[i], bias[i]));
                         float2 d2 = softplus ? softplus_fast2(r) : r;
                         if (!full_tile) {
-                            const bool ok0 = irow[i] >= 0 && (t0 + t + v0 + k) < p.L;
-                            const bool ok1 = irow[i] >= 0 && (t0 + t + v0 + k + 1) < p.L;
+                            const bool ok0 = irow[i] >= 0 && (t0 + t + v0 + k) < T1;
+                            const bool ok1 = irow[i] >= 0 && (t0 + t + v0 + k + 1) < T1;
                             d2 = make_float2(ok0 ? d2.x : 0.f, ok1 ? d2.y : 0.f);
                         } else if (irow[i] < 0) {
                             d2 = make_float2(0.f, 0.f);
@@ -515,7 +538,46 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                     float2 y2[4];
 #pragma unroll
                     for (int pp = 0; pp < 4; ++pp) y2[pp] = make_float2(0.f, 0.f);
-                    if constexpr (Ly::F32BC && !ZOH && !kPoly && kStepMajor) {
+                    if constexpr (kSummary) {
+                        // chunk summary: the recurrence alone (no readout);
+                        // with every A of the warp <= 0, the first
+                        // kSumPolyStates quarters of each lane's states take
+                        // their exponentials on the FMA pipe (ex2_poly2),
+                        // since this pass leaves issue slots free and the SFU
+                        // is the bound
+#pragma unroll
+                        for (int hb = 0; hb < 2; ++hb) {
+                            float4 Bv[NS];
+#pragma unroll
+                            for (int j = 0; j < NS; ++j) {
+                                if constexpr (Ly::F32BC) {
+                                    const int cc = (((tb >> 2) + hb) ^ bkey) << 2;
+                                    Bv[j] = *reinterpret_cast<const float4 *>(bcfB + j * TT + cc);
+                                } else {
+                                    float2 bq[4];
+                                    load_pairs8_at<T>(bc_chunk(rawB, rr0 + j, tb), bc_chunk(rawB, rr0 + j, tb + 4), bq);
+                                    Bv[j] = make_float4(bq[2 * hb].x, bq[2 * hb].y, bq[2 * hb + 1].x, bq[2 * hb + 1].y);
+                                }
+                            }
+#pragma unroll
+                            for (int pq = 0; pq < 2; ++pq) {
+                                const int pp = 2 * hb + pq;
+                                float2 a[NS], beta[NS];
+#pragma unroll
+                                for (int j = 0; j < NS; ++j) {
+                                    const float2 arg = __fmul2_rn(dtp[pp], A2d[j]);
+                                    if (kPoly && j < (NS * kSumPolyStates + 3) / 4)
+                                        a[j] = ex2_poly2(arg);
+                                    else
+                                        a[j] = make_float2(ex2(arg.x), ex2(arg.y));
+                                    const float2 bb = pq ? make_float2(Bv[j].z, Bv[j].w) : make_float2(Bv[j].x, Bv[j].y);
+                                    beta[j] = __fmul2_rn(dup[pp], bb);
+                                }
+#pragma unroll
+                                for (int j = 0; j < NS; ++j) h[j] = fmaf(a[j].y, fmaf(a[j].x, h[j], beta[j].x), beta[j].y);
+                            }
+                        }
+                    } else if constexpr (Ly::F32BC && !ZOH && !kPoly && kStepMajor) {
                         // step-major order: per pair of steps, every state's
                         // exponentials, then the NS independent recurrence
                         // chains side by side, then the readout
@@ -589,10 +651,12 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                         }
                     }
                     }
-                    *reinterpret_cast<float4 *>(myY + tb) = make_float4(y2[0].x, y2[0].y, y2[1].x, y2[1].y);
-                    *reinterpret_cast<float4 *>(myY + tb + 4) = make_float4(y2[2].x, y2[2].y, y2[3].x, y2[3].y);
+                    if constexpr (!kSummary) {
+                        *reinterpret_cast<float4 *>(myY + tb) = make_float4(y2[0].x, y2[0].y, y2[1].x, y2[1].y);
+                        *reinterpret_cast<float4 *>(myY + tb + 4) = make_float4(y2[2].x, y2[2].y, y2[3].x, y2[3].y);
+                    }
                     // checkpoint: the state after this 8-step block (a chunk)
-                    if (ck_row && t0 + tb < p.L) {
+                    if (ck_row && t0 + tb < T1) {
                         float *dst = ck_row + (size_t)((t0 + tb) / SSM_CKPT_CHUNK) * N;
 #pragma unroll
                         for (int j = 0; j < NS; ++j) dst[j] = h[j];
@@ -600,23 +664,23 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                 }
         
             };
-            if (kPolyPairs > 0 && poly_ok)
+            if ((kPolyPairs > 0 || (kSummary && kSumPolyStates > 0)) && poly_ok)
                 run_blocks(std::integral_constant<bool, true>{});
             else
                 run_blocks(std::integral_constant<bool, false>{});
             // the final state
             const int row = wrow0 + c;
-            if (live && p.last_state && tile == ntiles - 1) {
-                float *dst = p.last_state + (size_t)row * N + g * NS;
+            if (live && p.last_state && tile == ntiles - 1 && ((p.virt & 2) || kc == p.K - 1)) {
+                float *dst = p.last_state + (size_t)((p.virt & 2) ? voff + row : row) * N + g * NS;
 #pragma unroll
                 for (int j = 0; j < NS; ++j) dst[j] = h[j];
             }
             __syncwarp();
             // (3) Σ of the NT partials, D skip, gate, 16-byte stores
 #pragma unroll
-            for (int i = 0; i < IPL; ++i) {
+            for (int i = 0; i < (kSummary ? 0 : IPL); ++i) {
                 const int it = lane + 32 * i, rl = it / CPR, t = (it % CPR) * CHUNK;
-                if (irow[i] < 0 || t0 + t >= p.L) continue;
+                if (irow[i] < 0 || t0 + t >= T1) continue;
                 float y[CHUNK];
 #pragma unroll
                 for (int k = 0; k < CHUNK; k += 4) {
@@ -665,7 +729,7 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                 float v = dsum[i];
 #pragma unroll
                 for (int m = 1; m < CPR; m <<= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
-                if (irow[i] >= 0 && (lane % CPR) == 0) p.delta_sum[irow[i]] = v;
+                if (irow[i] >= 0 && (lane % CPR) == 0) p.delta_sum[(p.virt & 2) ? voff + irow[i] : irow[i]] = v;
             }
         }
         if (++tile == ntiles) { tile = 0; ++q; }
@@ -679,8 +743,13 @@ template <typename T, int NT, int NS, int TT, int NWC, int STAGES, int FL>
 cudaError_t launch_cfg(const FwdParams &fp, cudaStream_t stream) {
     using Ly = TmaLayout<T, NT, NS, TT, NWC, STAGES>;
     const int P = fp.batch * fp.dim;
-    const int grid = std::min(device_sm_count(), P);
-    const int R = (P + grid - 1) / grid;
+    const int K = std::max(1, fp.K);
+    const int grid = K > 1 ? device_sm_count() : std::min(device_sm_count(), P);
+    const int gk = grid / K;                      // fewest CTAs of a chunk
+    const int Lc = fp.Lc > 0 ? fp.Lc : fp.L;     // a chunk plan may cover less than L
+    if (gk < 1 || (fp.Lc > 0 && (Lc % TT != 0 || (long long)(K - 1) * Lc >= fp.L)))
+        return cudaErrorInvalidValue;   // chunks of whole tiles, each starting inside the sequence
+    const int R = (P + gk - 1) / gk;
     const int npass = (R + Ly::MAXR - 1) / Ly::MAXR;
     const int rows_max = (R + npass - 1) / npass;
     const bool bf16 = sizeof(T) == 2;
@@ -696,6 +765,7 @@ cudaError_t launch_cfg(const FwdParams &fp, cudaStream_t stream) {
     p.last_state = fp.last_state; p.ckpt = fp.ckpt; p.h0 = fp.h0; p.delta_sum = fp.delta_sum;
     p.P = P; p.dim = fp.dim; p.L = fp.L; p.n_ckpt = fp.n_ckpt;
     p.softplus = fp.softplus; p.has_z = fp.z != nullptr; p.rows_max = rows_max;
+    p.K = K; p.Lc = Lc; p.virt = fp.virt;
     p.err = device_error_word();
     if (!p.err) return cudaErrorInvalidDevice;
     auto kern = fwd_tma_kernel<T, NT, NS, TT, NWC, STAGES, FL>;
@@ -753,6 +823,9 @@ SSM_TMA_CFG(float, 8, 8, 8, 2)
 template <typename T, int N, int NT>
 cudaError_t launch_nt(const FwdParams &fp, cudaStream_t stream) {
     using C = TmaCfg<T, N, NT>;
+    if (fp.summary)
+        return fp.softplus ? launch_cfg<T, NT, N / NT, C::TT, C::NWC, C::STAGES, -3>(fp, stream)
+                           : launch_cfg<T, NT, N / NT, C::TT, C::NWC, C::STAGES, -4>(fp, stream);
     if constexpr (N == 16) {   // zero-order hold: dstate 16 only (else the general kernel)
         if (fp.zoh) return launch_cfg<T, NT, N / NT, C::TT, C::NWC, C::STAGES, -2>(fp, stream);
     }
@@ -809,20 +882,24 @@ bool nt_valid(int N, int nt) {
 // Returns true (and launches) when the TMA path applies; false means the
 // caller should use the general kernel.
 bool try_launch_fwd_tma(const FwdParams &fp, cudaStream_t stream, cudaError_t *err) {
-    if (!fp.vec_ok || !fp.out || (fp.zoh && fp.N != 16)) return false;   // ZOH: dstate 16 here
+    if (!fp.vec_ok || !(fp.out || fp.summary) || (fp.zoh && fp.N != 16)) return false;   // ZOH: dstate 16 here
+    if (fp.summary && fp.zoh) return false;
     if (fp.N != 8 && fp.N != 16 && fp.N != 32) return false;
     if (!tma_available()) return false;
     const long long P = (long long)fp.batch * fp.dim;
     const int sms = device_sm_count();
-    if (P < sms) return false;                      // fewer channels than SMs
-    const long long R = (P + sms - 1) / sms;        // rows per SM
+    const int K = std::max(1, fp.K);
+    const long long gk = sms / K;                   // fewest CTAs of a time chunk
+    if (gk < 1 || P < gk) return false;             // fewer channels than CTAs
+    const long long R = (P + gk - 1) / gk;          // rows per CTA
     // Lane split: the fewest lanes per channel that still give every SM
-    // 8 warps of lanes (more states per lane = less per-state overhead).
+    // 8 warps of lanes (more states per lane = less per-state overhead);
+    // chunk summaries, which carry no readout, settle for 4 warps.
     int nt = 0;
     for (int cand : {2, 4, 8, 16}) {
         if (!nt_valid(fp.N, cand)) continue;
         nt = cand;
-        if (R * cand >= 256) break;
+        if (R * cand >= (fp.summary ? 128 : 256)) break;
     }
     // SSM_TMA_NT overrides the lane split (tuning knob)
     static const char *force_nt = getenv("SSM_TMA_NT");
@@ -843,6 +920,114 @@ bool try_launch_fwd_tma(const FwdParams &fp, cudaStream_t stream, cudaError_t *e
     }
     *err = e;
     return true;
+}
+
+// ------------------------------------------------------------ two-level scan
+// For long sequences over few channel rows, one pass leaves most of each SM
+// idle: every (row, state) recurrence runs the whole length in one lane.  The
+// sequence is then cut into K chunks, and the chunks of a row run side by side
+// in three launches (booiljung.github.io, "3.2 선택적 스캔(Selective Scan)
+// 알고리즘", §2.2: the pairs (Ā, b) compose with (a_j, b_j) • (a_i, b_i) =
+// (a_j a_i, a_j b_i + b_j)):
+//  1. summaries of chunks 0..K-2: the end state e_k of each chunk run from a
+//     zero state, and Σ Δ over it (its decay product is exp(A Σ Δ));
+//  2. the exclusive combine of the summaries in sequence order: the state
+//     h_in[k] entering each chunk (launch_combine_carries);
+//  3. every chunk run again from h_in[k], writing the output.
+// Workspace: e [K-1][P][N], Σ Δ [K-1][P] (rounded up to 16 bytes), h_in
+// [K][P][N], all fp32.
+
+namespace {
+constexpr int kChunkMinSteps = 512;      // shortest chunk worth a pipeline fill
+size_t align16(size_t x) { return (x + 15) / 16 * 16; }
+
+// Modelled time of one launch over K chunks of Lc steps: the passes of its
+// busiest CTA times the warps on its busiest SM sub-partition times the
+// states each lane carries and the chunk length, weighted by the measured
+// cost per element-state of each lane split relative to 4 lanes per channel
+// (16 lanes 1.55x, from the long-context forward; 2 lanes 0.85x, from a
+// 128-row-per-SM chunked pass; 8 lanes taken as 1.3x).
+double launch_cost(long long P, int dim, long long K, long long Lc, int N, bool bf16, int sms,
+                   bool summary) {
+    const long long gk = sms / K;
+    if (gk < 1 || P < gk) return 1e300;        // a launch the TMA forward refuses
+    const long long R = (P + gk - 1) / gk;
+    int nt = 0;
+    for (int cand : {2, 4, 8, 16}) {
+        if (!nt_valid(N, cand)) continue;
+        nt = cand;
+        if (R * cand >= (summary ? 128 : 256)) break;
+    }
+    const long long cap = bf16 ? rows_cap<__nv_bfloat16>(N, nt) : rows_cap<float>(N, nt);
+    const long long npass = (R + cap - 1) / cap, rp = (R + npass - 1) / npass;
+    if (rp > dim) return 1e300;                 // a pass may touch at most two batch rows
+    const long long warps = (rp + 32 / nt - 1) / (32 / nt);
+    const double w = nt >= 16 ? 1.55 : nt == 8 ? 1.3 : nt == 2 ? 0.85 : 1.0;
+    return (double)npass * (double)((warps + 3) / 4) * (N / nt) * (double)Lc * w;
+}
+}  // namespace
+
+// The chunk plan: the K (and chunk length, whole 128-step blocks) that
+// minimises the modelled time of the two-level scan (a summary pass counted at
+// 0.7 of a full pass), taken only when that is below 0.85 of the one-pass
+// forward's modelled time.  SSM_FWD_CHUNKS=K in the environment forces K.
+size_t fwd_chunk_plan(const FwdParams &fp, int *Kp, int *Lcp) {
+    if (!fp.vec_ok || fp.zoh || fp.delta_sum) return 0;
+    if (fp.N != 8 && fp.N != 16 && fp.N != 32) return 0;
+    if (!tma_available()) return 0;
+    const long long P = (long long)fp.batch * fp.dim;
+    const int sms = device_sm_count();
+    if (sms < 2) return 0;
+    static const char *force = getenv("SSM_FWD_CHUNKS");
+    const long long forced = force ? atoll(force) : 0;
+    long long bestK = 0, bestLc = 0;
+    double best = 0.85 * launch_cost(P, fp.dim, 1, fp.L, fp.N, fp.io_bf16, sms, false);
+    const long long kmax = std::min<long long>(sms, fp.L / kChunkMinSteps);
+    for (long long K = 2; K <= kmax; ++K) {
+        const long long Lc = ((fp.L + K - 1) / K + 127) / 128 * 128;
+        const long long K2 = (fp.L + Lc - 1) / Lc;
+        if (K2 < 2 || (forced >= 2 && K != forced)) continue;
+        const double c = launch_cost(P, fp.dim, K2, Lc, fp.N, fp.io_bf16, sms, false) +
+                         0.7 * launch_cost(P, fp.dim, K2 - 1, Lc, fp.N, fp.io_bf16, sms, true);
+        if (c < best || (forced >= 2 && !bestK && c < 1e299)) {
+            best = c;
+            bestK = K2;
+            bestLc = Lc;
+        }
+    }
+    if (bestK < 2) return 0;
+    if (Kp) *Kp = (int)bestK;
+    if (Lcp) *Lcp = (int)bestLc;
+    const size_t PN = (size_t)P * fp.N * sizeof(float);
+    return (size_t)(bestK - 1) * PN + align16((size_t)(bestK - 1) * P * sizeof(float)) +
+           (size_t)bestK * PN;
+}
+
+cudaError_t launch_fwd_chunked(const FwdParams &fp, void *ws, size_t ws_bytes, cudaStream_t stream) {
+    int K = 0, Lc = 0;
+    const size_t need = fwd_chunk_plan(fp, &K, &Lc);
+    if (need == 0 || ws_bytes < need || !ws || (reinterpret_cast<uintptr_t>(ws) & 15)) return cudaErrorInvalidValue;
+    const long long P = (long long)fp.batch * fp.dim;
+    float *h_ends = static_cast<float *>(ws);
+    float *dsums = h_ends + (size_t)(K - 1) * P * fp.N;
+    float *h_in = reinterpret_cast<float *>(reinterpret_cast<char *>(dsums) +
+                                           align16((size_t)(K - 1) * P * sizeof(float)));
+    cudaError_t e = cudaSuccess;
+    // 1. summaries of chunks 0..K-2 (end states from zero, Σ Δ), per virtual row
+    FwdParams s = fp;
+    s.out = nullptr; s.z = nullptr; s.ckpt = nullptr; s.h0 = nullptr;
+    s.last_state = h_ends; s.delta_sum = dsums;
+    s.K = K - 1; s.Lc = Lc; s.virt = 2; s.summary = true;
+    if (!try_launch_fwd_tma(s, stream, &e)) return cudaErrorNotSupported;
+    if (e != cudaSuccess) return e;
+    // 2. the state entering each chunk (the caller's h0 enters chunk 0)
+    e = launch_combine_carries(K, P, fp.dim, fp.N, fp.A, dsums, h_ends, fp.h0, h_in, stream);
+    if (e != cudaSuccess) return e;
+    // 3. every chunk from its carry-in; last_state from the last chunk
+    FwdParams f = fp;
+    f.h0 = h_in; f.K = K; f.Lc = Lc; f.virt = 1; f.summary = false;
+    if (!try_launch_fwd_tma(f, stream, &e)) return cudaErrorNotSupported;
+    return e;
 }
 
 }  // namespace ssm

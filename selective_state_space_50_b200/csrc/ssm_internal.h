@@ -25,6 +25,13 @@ struct FwdParams {
     int zoh;      // zero-order-hold B̄ (general kernels only)
     bool io_bf16;
     bool vec_ok;  // every [.., L] row starts 16-byte aligned
+    // Two-level scan along L (TMA forward only): K time chunks of Lc steps
+    // (K <= 1: one pass over the whole sequence), `virt` bits as in the
+    // kernel (1: h0 per chunk and row; 2: last_state / delta_sum per chunk
+    // and row), `summary`: chunk summaries only (end state from h = 0 and
+    // Σ Δ; no output).
+    int K, Lc, virt;
+    bool summary;
 };
 
 struct BwdParams {
@@ -84,6 +91,12 @@ enum class FwdKernel { kAuto = 0, kGeneral = 1, kTma = 2 };
 FwdKernel fwd_kernel_choice();
 
 cudaError_t launch_fwd(const FwdParams &p, bool states_only, cudaStream_t stream);
+// The chunked two-level forward for long sequences over few channel rows:
+// fwd_chunk_plan returns the workspace bytes it needs (0: the shape is better
+// served by one pass), launch_fwd_chunked runs it (summaries, carry combine,
+// full pass from the carries) in `ws`.
+size_t fwd_chunk_plan(const FwdParams &p, int *K, int *Lc);
+cudaError_t launch_fwd_chunked(const FwdParams &p, void *ws, size_t ws_bytes, cudaStream_t stream);
 // Launches the TMA-fed persistent forward when it applies (returns true and
 // sets *err); returns false when the general kernel must be used.
 bool try_launch_fwd_tma(const FwdParams &p, cudaStream_t stream, cudaError_t *err);

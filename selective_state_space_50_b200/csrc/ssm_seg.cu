@@ -70,7 +70,9 @@ __global__ void __launch_bounds__(256) combine_kernel(int nseg, long long P, int
     float h = h0 ? h0[i] : 0.f;
     for (int s = 0; s < nseg; ++s) {
         h_in[(long long)s * P * N + i] = h;
-        h = fmaf(exp2f(a2 * dsums[(long long)s * P + row]), h, h_ends[(long long)s * P * N + i]);
+        // the last segment's summary is not needed (and may be absent)
+        if (s + 1 < nseg)
+            h = fmaf(exp2f(a2 * dsums[(long long)s * P + row]), h, h_ends[(long long)s * P * N + i]);
     }
 }
 

@@ -29,7 +29,8 @@ EXPORTS = ("ssm_version", "ssm_last_error_string", "ssm_selective_scan_ckpt_byte
            "ssm_selective_scan_fwd_ex", "ssm_selective_scan_bwd_ex",
            "ssm_selective_state_update_ex", "ssm_selftest_wait_timeout",
            "ssm_selection_projections", "ssm_selective_scan_fwd_segment",
-           "ssm_scan_combine_carries")
+           "ssm_scan_combine_carries", "ssm_selective_scan_fwd_workspace_bytes",
+           "ssm_selective_scan_fwd_ws")
 SSM_DISC_DELTA_B, SSM_DISC_ZOH = 0, 1
 NOALLOC_SCRATCH_BYTES = 32 << 20  # SSM_NOALLOC_SCRATCH_BYTES in include/ssm_scan.h
 
@@ -86,6 +87,10 @@ def load_library(path: str = LIB_PATH):
     op = ctypes.POINTER(Options)
     lib.ssm_selective_scan_fwd_ex.argtypes = [sp, op] + [vp] * 12
     lib.ssm_selective_scan_fwd_ex.restype = i
+    lib.ssm_selective_scan_fwd_workspace_bytes.argtypes = [sp, op, ctypes.POINTER(sz)]
+    lib.ssm_selective_scan_fwd_workspace_bytes.restype = i
+    lib.ssm_selective_scan_fwd_ws.argtypes = [sp, op] + [vp] * 12 + [sz, vp]
+    lib.ssm_selective_scan_fwd_ws.restype = i
     lib.ssm_selective_scan_bwd_ex.argtypes = [sp, op] + [vp] * 19 + [sz, vp]
     lib.ssm_selective_scan_bwd_ex.restype = i
     lib.ssm_selective_state_update_ex.argtypes = [sp, op] + [vp] * 11
@@ -151,10 +156,29 @@ def _shape_of(u: torch.Tensor, A: torch.Tensor) -> Shape:
     return make_shape(u.shape[0], u.shape[1], u.shape[2], A.shape[1], u.dtype)
 
 
+def fwd_workspace_bytes(shape: Shape, delta_softplus: bool = True, zoh: bool = False) -> int:
+    """Workspace bytes of ssm_selective_scan_fwd_ws for this shape on the
+    current device (0: the one-pass forward, no workspace needed)."""
+    n = ctypes.c_size_t()
+    o = _opts(delta_softplus, zoh)
+    _check(load_library().ssm_selective_scan_fwd_workspace_bytes(ctypes.byref(shape), ctypes.byref(o),
+                                                                 ctypes.byref(n)))
+    return int(n.value)
+
+
 def fwd_raw(shape: Shape, u, delta, A, B, C, D, z, delta_bias, delta_softplus: bool,
-            out, last_state, ckpt, stream=None, zoh: bool = False):
+            out, last_state, ckpt, stream=None, zoh: bool = False, workspace=None):
     """Direct C-ABI call on raw tensors (no checks beyond the library's own).
-    zoh selects the zero-order-hold B̄ (ssm_selective_scan_fwd_ex)."""
+    zoh selects the zero-order-hold B̄ (ssm_selective_scan_fwd_ex); a
+    workspace tensor selects ssm_selective_scan_fwd_ws (the two-level scan
+    along the sequence where the shape calls for it)."""
+    if workspace is not None:
+        o = _opts(delta_softplus, zoh)
+        _check(load_library().ssm_selective_scan_fwd_ws(
+            ctypes.byref(shape), ctypes.byref(o), _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C),
+            _ptr(D), _ptr(z), _ptr(delta_bias), _ptr(out), _ptr(last_state), _ptr(ckpt),
+            _ptr(workspace), workspace.numel() * workspace.element_size(), _stream_ptr(stream)))
+        return
     if zoh:
         o = _opts(delta_softplus, True)
         _check(load_library().ssm_selective_scan_fwd_ex(
@@ -249,7 +273,10 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None,
                         dtype=torch.float32) if return_last_state else None)
     ck = (torch.empty(ckpt_numel(shape), device=u.device, dtype=torch.float32)
           if return_ckpt else None)
-    fwd_raw(shape, u, delta, A, B, C, D, z, delta_bias, delta_softplus, out, last, ck, stream, zoh)
+    nws = fwd_workspace_bytes(shape, delta_softplus, zoh)
+    ws = torch.empty(nws // 4, device=u.device, dtype=torch.float32) if nws else None
+    fwd_raw(shape, u, delta, A, B, C, D, z, delta_bias, delta_softplus, out, last, ck, stream, zoh,
+            workspace=ws)
     return out, last, ck
 
 
