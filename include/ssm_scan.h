@@ -102,6 +102,15 @@ int ssm_version(void);
 const char *ssm_last_error_string(void);
 
 /*
+ * Diagnostic (the pages have no counterpart): which kernels the last forward
+ * or backward call on this thread launched: "fwd:tma", "fwd:general",
+ * "fwd:chunked" (the two-level scan of ssm_selective_scan_fwd_ws), "bwd:tma"
+ * or "bwd:general" ("" before any call).  A static string; the library owns
+ * it.
+ */
+const char *ssm_last_kernel_path(void);
+
+/*
  * Bytes of the optional checkpoint buffer `ckpt` of ssm_selective_scan_fwd:
  * batch * dim * ceil(seqlen / SSM_CKPT_CHUNK) * dstate * 4.
  */

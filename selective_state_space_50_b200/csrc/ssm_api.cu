@@ -40,6 +40,7 @@ cudaError_t read_and_clear_device_error(int *value, cudaStream_t stream) {
 namespace {
 
 thread_local std::string g_last_error;
+thread_local const char *g_kernel_path = "";
 
 ssm_status_t fail(ssm_status_t st, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
 ssm_status_t fail(ssm_status_t st, const char *fmt, ...) {
@@ -129,6 +130,8 @@ ssm_status_t check_options(const ssm_options_t *o) {
 
 }  // namespace
 
+void ssm::set_kernel_path(const char *path) { g_kernel_path = path ? path : ""; }
+
 ssm_status_t ssm::set_last_error(ssm_status_t status, const char *msg) {
     g_last_error = msg ? msg : "";
     return status;
@@ -139,6 +142,8 @@ extern "C" {
 int ssm_version(void) { return 100; }
 
 const char *ssm_last_error_string(void) { return g_last_error.c_str(); }
+
+const char *ssm_last_kernel_path(void) { return g_kernel_path; }
 
 ssm_status_t ssm_selective_scan_ckpt_bytes(const ssm_shape_t *shape, size_t *bytes) {
     SSM_TRY(check_shape(shape));

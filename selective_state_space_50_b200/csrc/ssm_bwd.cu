@@ -360,7 +360,11 @@ static cudaError_t launch_bwd_t(const BwdParams &p, cudaStream_t stream) {
 
 cudaError_t launch_bwd(const BwdParams &p, cudaStream_t stream) {
     cudaError_t err = cudaSuccess;
-    if (try_launch_bwd_tma(p, stream, &err)) return err;
+    if (try_launch_bwd_tma(p, stream, &err)) {
+        set_kernel_path("bwd:tma");
+        return err;
+    }
+    set_kernel_path("bwd:general");
     return p.io_bf16 ? launch_bwd_t<__nv_bfloat16>(p, stream) : launch_bwd_t<float>(p, stream);
 }
 

@@ -149,7 +149,11 @@ __device__ __forceinline__ float group_reduce4(float2 p01, float2 p23, int g) {
 
 // ALN: the channel count is a multiple of 8 and CTAs and passes start on
 // multiples of 8 rows, so that no warp's 8 channels span two batch rows.
-template <typename T, int NWC, int STAGES, bool HZ, bool SP, bool ALN>
+// ZOH: zero-order hold, B̄ = φ(Δ A) Δ B with φ(x) = (e^x - 1)/x
+// (booiljung.github.io, "3.2 선택적 스캔(Selective Scan) 알고리즘" §2.1), whose
+// derivatives are d(φ Δ)/dΔ = Ā and d(φ Δ)/dA = Δ² ψ(Δ A); φ and ψ come from
+// Ā, 1/Δ and 1/A (zoh_phi2, zoh_psi2), with no division per element-state.
+template <typename T, int NWC, int STAGES, bool HZ, bool SP, bool ALN, bool ZOH>
 __global__ void __launch_bounds__((NWC + 1) * 32, 1)
 bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constant__ CUtensorMap m_u,
                const __grid_constant__ CUtensorMap m_z, const __grid_constant__ CUtensorMap m_g,
@@ -332,6 +336,7 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
     float *myX = wX + lane * XS;
 
     float2 A2p[NS], dA2[NS];                                   // (A log2 e) twice; dA partials
+    float2 iA2[NS];                                            // 1 / A twice (zero-order hold)
     float lam[NS], anext[NS];
     float4 hpre = make_float4(0.f, 0.f, 0.f, 0.f);             // checkpoint of the next window
     float dD_acc = 0.f, db_acc = 0.f, Dd = 0.f, bias_c = 0.f, i_bias = 0.f;
@@ -355,8 +360,13 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
             wb = b1mask != 0 ? 1 : 0;
 #pragma unroll
             for (int j = 0; j < NS; ++j) {
-                const float a2 = live ? p.A[(size_t)d * N + g * NS + j] * SSM_LOG2E : 0.f;
+                const float av = live ? p.A[(size_t)d * N + g * NS + j] : 0.f;
+                const float a2 = av * SSM_LOG2E;
                 A2p[j] = make_float2(a2, a2);
+                if constexpr (ZOH) {
+                    const float ia = 1.f / av;
+                    iA2[j] = make_float2(ia, ia);
+                }
                 dA2[j] = make_float2(0.f, 0.f);
                 lam[j] = 0.f;
                 anext[j] = 1.f;
@@ -487,7 +497,7 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                 float2 ab2[W / 2][NS], ahp2[W / 2][NS];
                 // per half-window, summed over the state groups: y, Σ λ A Ā h
                 // (units of A log2 e) and Σ λ B at step 4 hh + g of channel c
-                float yv[2], sav[2], sbv[2];
+                float yv[2], sav[2], sbv[2], sqv[2];
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     const int tb = tw + 4 * hh;
@@ -497,6 +507,12 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                     const float2 dtp[2] = {make_float2(dt4.x, dt4.y), make_float2(dt4.z, dt4.w)};
                     const float2 dup[2] = {make_float2(du4.x, du4.y), make_float2(du4.z, du4.w)};
                     const float2 gyp[2] = {make_float2(gy4.x, gy4.y), make_float2(gy4.z, gy4.w)};
+                    float2 idt[2];                          // 1/Δ (zero-order hold)
+                    if constexpr (ZOH) {
+#pragma unroll
+                        for (int pp = 0; pp < 2; ++pp)
+                            idt[pp] = make_float2(rcp_approx(dtp[pp].x), rcp_approx(dtp[pp].y));
+                    }
                     float2 y2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
                     for (int j = 0; j < NS; ++j) {
@@ -509,7 +525,8 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                             const int P = 2 * hh + pp;
                             const float2 arg = __fmul2_rn(dtp[pp], A2p[j]);
                             const float2 a = make_float2(ex2(arg.x), ex2(arg.y));
-                            const float2 beta = __fmul2_rn(dup[pp], Bp[pp]);
+                            float2 beta = __fmul2_rn(dup[pp], Bp[pp]);
+                            if constexpr (ZOH) beta = __fmul2_rn(beta, zoh_phi2(arg, a, idt[pp], iA2[j]));
                             const float h0 = fmaf(a.x, h[j], beta.x);
                             const float h1 = fmaf(a.y, h0, beta.y);
                             h[j] = h1;
@@ -538,6 +555,14 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                     const float2 gyp[2] = {make_float2(gy4.x, gy4.y), make_float2(gy4.z, gy4.w)};
                     float2 sa2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
                     float2 sb2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+                    // zero-order hold: Σ λ B Ā (the B term of dΔ); sb2 holds Σ λ B φ
+                    float2 sq2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+                    float2 idt[2];
+                    if constexpr (ZOH) {
+#pragma unroll
+                        for (int pp = 0; pp < 2; ++pp)
+                            idt[pp] = make_float2(rcp_approx(dtp[pp].x), rcp_approx(dtp[pp].y));
+                    }
 #pragma unroll
                     for (int j = 0; j < NS; ++j) {
                         const float4 B4 = bc4(bcfB, j, tb), C4 = bc4(bcfC, j, tb);
@@ -552,10 +577,24 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                             const float l0 = fmaf(ab2[P][j].y, l1, cg.x);       // λ of the earlier step
                             const float2 l2 = make_float2(l0, l1);
                             const float2 wv = __fmul2_rn(l2, ahp2[P][j]);
-                            dA2[j] = __ffma2_rn(dtp[pp], wv, dA2[j]);
                             sa2[pp] = __ffma2_rn(A2p[j], wv, sa2[pp]);
-                            sb2[pp] = __ffma2_rn(l2, Bp[pp], sb2[pp]);
-                            xb[pp] = __fmul2_rn(l2, dup[pp]);
+                            if constexpr (ZOH) {
+                                // β = φ Δ B u: dβ/dΔ = Ā B u, dβ/dA = Δ² ψ B u,
+                                // dβ/du = φ Δ B, dβ/dB = φ Δ u
+                                const float2 arg = __fmul2_rn(dtp[pp], A2p[j]);
+                                const float2 phi = zoh_phi2(arg, ab2[P][j], idt[pp], iA2[j]);
+                                const float2 psi = zoh_psi2(arg, ab2[P][j], phi, idt[pp], iA2[j]);
+                                const float2 lB = __fmul2_rn(l2, Bp[pp]);
+                                sb2[pp] = __ffma2_rn(lB, phi, sb2[pp]);
+                                sq2[pp] = __ffma2_rn(lB, ab2[P][j], sq2[pp]);
+                                const float2 w2 = __ffma2_rn(lB, __fmul2_rn(dup[pp], psi), wv);
+                                dA2[j] = __ffma2_rn(dtp[pp], w2, dA2[j]);
+                                xb[pp] = __fmul2_rn(__fmul2_rn(l2, dup[pp]), phi);
+                            } else {
+                                dA2[j] = __ffma2_rn(dtp[pp], wv, dA2[j]);
+                                sb2[pp] = __ffma2_rn(l2, Bp[pp], sb2[pp]);
+                                xb[pp] = __fmul2_rn(l2, dup[pp]);
+                            }
                             lam[j] = l0;
                             anext[j] = ab2[P][j].x;
                         }
@@ -564,6 +603,7 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                     }
                     sav[hh] = group_reduce4(sa2[0], sa2[1], g);
                     sbv[hh] = group_reduce4(sb2[0], sb2[1], g);
+                    if constexpr (ZOH) sqv[hh] = group_reduce4(sq2[0], sq2[1], g);
                 }
                 reduce_x(0, tw);
                 // per-element results: lane (g, c) finishes steps g and g + 4 of channel c
@@ -584,7 +624,7 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                             const float sg = sigmoid(zz);
                             __stcs(p.dz + off, gv * yy * sg * fmaf(zz, 1.f - sg, 1.f));
                         }
-                        const float dDelta = fmaf(x, sb, sa);
+                        const float dDelta = fmaf(x, ZOH ? sqv[e] : sb, sa);
                         const float ddv = SP ? dDelta * sigmoid(IO<T>::to_f(rawD[o]) + bias_c) : dDelta;
                         __stcs(p.du + off, fmaf(gyv, Dd, dtv * sb));
                         __stcs(p.ddelta + off, ddv);
@@ -625,7 +665,7 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
 // ------------------------------------------------------------------ host side
 
 
-template <typename T, int NWC, int STAGES, bool HZ, bool SP, bool ALN>
+template <typename T, int NWC, int STAGES, bool HZ, bool SP, bool ALN, bool ZOH>
 cudaError_t launch_bwd_tma_cfg(const BwdParams &bp, int rows_max, cudaStream_t stream) {
     using Ly = BwdLayout<T, NWC, STAGES>;
     const int P = bp.batch * bp.dim;
@@ -648,7 +688,7 @@ cudaError_t launch_bwd_tma_cfg(const BwdParams &bp, int rows_max, cudaStream_t s
     p.softplus = bp.softplus; p.has_z = bp.z != nullptr; p.rows_max = rows_max;
     p.err = device_error_word();
     if (!p.err) return cudaErrorInvalidDevice;
-    auto kern = bwd_tma_kernel<T, NWC, STAGES, HZ, SP, ALN>;
+    auto kern = bwd_tma_kernel<T, NWC, STAGES, HZ, SP, ALN, ZOH>;
     static bool attr_done = false;
     if (!attr_done) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Ly::kAlloc);
@@ -665,22 +705,25 @@ cudaError_t launch_bwd_tma_cfg(const BwdParams &bp, int rows_max, cudaStream_t s
 #endif
 constexpr int kBwdStages = SSM_BWD_STAGES;
 
-// The gate, the softplus and the 8-row alignment are compile-time switches
-// of the kernel.
-template <typename T, int NWC, bool ALN>
+// The gate, the softplus, the 8-row alignment and the discretisation are
+// compile-time switches of the kernel.
+template <typename T, int NWC, bool ALN, bool ZOH>
 cudaError_t launch_bwd_tma_flags(const BwdParams &bp, int rows_max, cudaStream_t stream) {
     const bool hz = bp.z != nullptr, sp = bp.softplus != 0;
     constexpr int S = kBwdStages;
-    if (hz && sp) return launch_bwd_tma_cfg<T, NWC, S, true, true, ALN>(bp, rows_max, stream);
-    if (hz) return launch_bwd_tma_cfg<T, NWC, S, true, false, ALN>(bp, rows_max, stream);
-    if (sp) return launch_bwd_tma_cfg<T, NWC, S, false, true, ALN>(bp, rows_max, stream);
-    return launch_bwd_tma_cfg<T, NWC, S, false, false, ALN>(bp, rows_max, stream);
+    if (hz && sp) return launch_bwd_tma_cfg<T, NWC, S, true, true, ALN, ZOH>(bp, rows_max, stream);
+    if (hz) return launch_bwd_tma_cfg<T, NWC, S, true, false, ALN, ZOH>(bp, rows_max, stream);
+    if (sp) return launch_bwd_tma_cfg<T, NWC, S, false, true, ALN, ZOH>(bp, rows_max, stream);
+    return launch_bwd_tma_cfg<T, NWC, S, false, false, ALN, ZOH>(bp, rows_max, stream);
 }
 
 template <typename T, int NWC>
 cudaError_t launch_bwd_tma_aln(const BwdParams &bp, int rows_max, bool aln, cudaStream_t stream) {
-    return aln ? launch_bwd_tma_flags<T, NWC, true>(bp, rows_max, stream)
-               : launch_bwd_tma_flags<T, NWC, false>(bp, rows_max, stream);
+    if (bp.zoh)
+        return aln ? launch_bwd_tma_flags<T, NWC, true, true>(bp, rows_max, stream)
+                   : launch_bwd_tma_flags<T, NWC, false, true>(bp, rows_max, stream);
+    return aln ? launch_bwd_tma_flags<T, NWC, true, false>(bp, rows_max, stream)
+               : launch_bwd_tma_flags<T, NWC, false, false>(bp, rows_max, stream);
 }
 
 bool aligned_to(const void *ptr, uintptr_t a) { return (reinterpret_cast<uintptr_t>(ptr) % a) == 0; }
@@ -701,7 +744,7 @@ constexpr int kBwdWarpsBf16 = SSM_BWD_WARPS_BF16, kBwdWarpsF32 = SSM_BWD_WARPS_F
 bool try_launch_bwd_tma(const BwdParams &bp, cudaStream_t stream, cudaError_t *err) {
     static const char *force = getenv("SSM_BWD_KERNEL");
     if (force && !strcmp(force, "general")) return false;
-    if (!bp.vec_ok || bp.N != 16 || !bp.ckpt || bp.zoh) return false;   // zero-order hold: general kernel
+    if (!bp.vec_ok || bp.N != 16 || !bp.ckpt) return false;
     if (!aligned_to(bp.ckpt, 16) || !aligned_to(bp.dB, 16) || !aligned_to(bp.dC, 16) ||
         !aligned_to(bp.du, 8) || !aligned_to(bp.ddelta, 8) || (bp.dz && !aligned_to(bp.dz, 8)))
         return false;

@@ -124,6 +124,57 @@ __device__ __forceinline__ float zoh_psi(float x, float a) {
     return __fdividef(fmaf(x, a, 1.f - a), x * x);
 }
 
+// Zero-order-hold factor φ = (Ā - 1)/(Δ A) for a pair of steps of one state,
+// with arg = Δ A log2(e), a = 2^arg = Ā, idt = 1/Δ per step and ia = 1/A:
+// (a - 1) · idt · ia, or, for |Δ A| < 0.1 where a - 1 cancels, the Taylor
+// series 1 + x/2 + x²/6 + x³/24 + x⁴/120 + x⁵/720 in x = arg ln 2 (its
+// coefficients below are pre-scaled by powers of ln 2, so it runs in arg).
+// Exact zeros (Δ = 0 or A = 0) take the series: φ = 1, the Δ·B limit.
+__device__ __forceinline__ float2 zoh_phi2(float2 arg, float2 a, float2 idt, float2 ia) {
+    constexpr float L1 = 0.34657359f;      // ln2 / 2
+    constexpr float L2 = 0.080075502f;     // ln2^2 / 6
+    constexpr float L3 = 0.013876027f;     // ln2^3 / 24
+    constexpr float L4 = 0.0019236258f;    // ln2^4 / 120
+    constexpr float L5 = 0.00022222597f;   // ln2^5 / 720
+    float2 ser = __ffma2_rn(arg, make_float2(L5, L5), make_float2(L4, L4));
+    ser = __ffma2_rn(arg, ser, make_float2(L3, L3));
+    ser = __ffma2_rn(arg, ser, make_float2(L2, L2));
+    ser = __ffma2_rn(arg, ser, make_float2(L1, L1));
+    ser = __ffma2_rn(arg, ser, make_float2(1.f, 1.f));
+    const float2 em1 = __fadd2_rn(a, make_float2(-1.f, -1.f));
+    const float2 q = __fmul2_rn(__fmul2_rn(em1, idt), ia);
+    constexpr float kSmall = 0.14426950f;  // |Δ A| < 0.1  <=>  |arg| < 0.1 log2(e)
+    return make_float2(fabsf(arg.x) < kSmall ? ser.x : q.x, fabsf(arg.y) < kSmall ? ser.y : q.y);
+}
+
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// ψ = (Ā - φ)/(Δ A) for a pair of steps of one state (the factor of Δ² in the
+// derivative of the zero-order-hold input matrix with respect to A, with
+// ψ(x) = (x e^x - (e^x - 1))/x²), in the same units as zoh_phi2: arg = Δ A
+// log2(e), a = Ā, phi = φ, idt = 1/Δ, ia = 1/A.  For |Δ A| < 0.1, where
+// Ā - φ cancels, its Taylor series 1/2 + x/3 + x²/8 + x³/30 + x⁴/144 in
+// x = arg ln 2 (coefficients pre-scaled by powers of ln 2; truncation below
+// 2e-8).  Exact zeros (Δ = 0 or A = 0) take the series: ψ = 1/2.
+__device__ __forceinline__ float2 zoh_psi2(float2 arg, float2 a, float2 phi, float2 idt, float2 ia) {
+    constexpr float M1 = 0.23104906f;      // ln2 / 3
+    constexpr float M2 = 0.060056627f;     // ln2^2 / 8
+    constexpr float M3 = 0.011100822f;     // ln2^3 / 30
+    constexpr float M4 = 0.0016030215f;    // ln2^4 / 144
+    float2 ser = __ffma2_rn(arg, make_float2(M4, M4), make_float2(M3, M3));
+    ser = __ffma2_rn(arg, ser, make_float2(M2, M2));
+    ser = __ffma2_rn(arg, ser, make_float2(M1, M1));
+    ser = __ffma2_rn(arg, ser, make_float2(0.5f, 0.5f));
+    const float2 d = __fadd2_rn(a, make_float2(-phi.x, -phi.y));
+    const float2 q = __fmul2_rn(__fmul2_rn(d, idt), ia);
+    constexpr float kSmallPsi = 0.14426950f;  // |Δ A| < 0.1
+    return make_float2(fabsf(arg.x) < kSmallPsi ? ser.x : q.x, fabsf(arg.y) < kSmallPsi ? ser.y : q.y);
+}
+
 // ---- io element types -------------------------------------------------------
 
 template <typename T> struct IO;

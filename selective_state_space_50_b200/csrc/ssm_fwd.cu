@@ -307,9 +307,13 @@ cudaError_t launch_fwd(const FwdParams &p, bool states_only, cudaStream_t stream
     const FwdKernel choice = fwd_kernel_choice();
     if (!states_only && choice != FwdKernel::kGeneral) {
         cudaError_t e = cudaSuccess;
-        if (try_launch_fwd_tma(p, stream, &e)) return e;   // also writes delta_sum
+        if (try_launch_fwd_tma(p, stream, &e)) {   // also writes delta_sum
+            set_kernel_path("fwd:tma");
+            return e;
+        }
         if (choice == FwdKernel::kTma) return cudaErrorNotSupported;
     }
+    set_kernel_path(states_only ? "fwd:general-states" : "fwd:general");
     cudaError_t e;
     if (p.io_bf16)
         e = states_only ? launch_fwd_t<__nv_bfloat16, 1>(p, stream)

@@ -177,35 +177,6 @@ __device__ __forceinline__ void load_pairs8_at<float>(const float *lo, const flo
     v[2] = make_float2(b.x, b.y); v[3] = make_float2(b.z, b.w);
 }
 
-// Zero-order-hold factor φ = (Ā - 1)/(Δ A) for a pair of steps of one state,
-// with arg = Δ A log2(e), a = 2^arg = Ā, idt = 1/Δ per step and ia = 1/A:
-// (a - 1) · idt · ia, or, for |Δ A| < 0.1 where a - 1 cancels, the Taylor
-// series 1 + x/2 + x²/6 + x³/24 + x⁴/120 + x⁵/720 in x = arg ln 2 (its
-// coefficients below are pre-scaled by powers of ln 2, so it runs in arg).
-// Exact zeros (Δ = 0 or A = 0) take the series: φ = 1, the Δ·B limit.
-__device__ __forceinline__ float2 zoh_phi2(float2 arg, float2 a, float2 idt, float2 ia) {
-    constexpr float L1 = 0.34657359f;      // ln2 / 2
-    constexpr float L2 = 0.080075502f;     // ln2^2 / 6
-    constexpr float L3 = 0.013876027f;     // ln2^3 / 24
-    constexpr float L4 = 0.0019236258f;    // ln2^4 / 120
-    constexpr float L5 = 0.00022222597f;   // ln2^5 / 720
-    float2 ser = __ffma2_rn(arg, make_float2(L5, L5), make_float2(L4, L4));
-    ser = __ffma2_rn(arg, ser, make_float2(L3, L3));
-    ser = __ffma2_rn(arg, ser, make_float2(L2, L2));
-    ser = __ffma2_rn(arg, ser, make_float2(L1, L1));
-    ser = __ffma2_rn(arg, ser, make_float2(1.f, 1.f));
-    const float2 em1 = __fadd2_rn(a, make_float2(-1.f, -1.f));
-    const float2 q = __fmul2_rn(__fmul2_rn(em1, idt), ia);
-    constexpr float kSmall = 0.14426950f;  // |Δ A| < 0.1  <=>  |arg| < 0.1 log2(e)
-    return make_float2(fabsf(arg.x) < kSmall ? ser.x : q.x, fabsf(arg.y) < kSmall ? ser.y : q.y);
-}
-
-__device__ __forceinline__ float rcp_approx(float x) {
-    float y;
-    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
 // FL >= 0: the gate, softplus and checkpoint options are compile-time bits
 // (1: gate z, 2: softplus, 4: checkpoints); B̄ = Δ B.  FL = -1: the options
 // are read at run time; B̄ = Δ B.  FL = -2: options at run time, zero-order
@@ -1027,6 +998,7 @@ cudaError_t launch_fwd_chunked(const FwdParams &fp, void *ws, size_t ws_bytes, c
     FwdParams f = fp;
     f.h0 = h_in; f.K = K; f.Lc = Lc; f.virt = 1; f.summary = false;
     if (!try_launch_fwd_tma(f, stream, &e)) return cudaErrorNotSupported;
+    set_kernel_path("fwd:chunked");
     return e;
 }
 

@@ -100,6 +100,10 @@ cudaError_t launch_fwd_chunked(const FwdParams &p, void *ws, size_t ws_bytes, cu
 // Launches the TMA-fed persistent forward when it applies (returns true and
 // sets *err); returns false when the general kernel must be used.
 bool try_launch_fwd_tma(const FwdParams &p, cudaStream_t stream, cudaError_t *err);
+// Records which kernels the last launch on this thread used (the string
+// behind ssm_last_kernel_path; a static string literal).
+void set_kernel_path(const char *path);
+
 // Records `msg` as this thread's last error (ssm_last_error_string) and
 // returns `status`.
 ssm_status_t set_last_error(ssm_status_t status, const char *msg);

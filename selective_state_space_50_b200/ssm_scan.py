@@ -22,7 +22,8 @@ SSM_OK, SSM_ERR_INVALID_ARG, SSM_ERR_UNSUPPORTED, SSM_ERR_CUDA, SSM_ERR_TIMEOUT 
 SSM_F32, SSM_BF16 = 0, 1
 CKPT_CHUNK = 8  # SSM_CKPT_CHUNK in include/ssm_scan.h
 
-EXPORTS = ("ssm_version", "ssm_last_error_string", "ssm_selective_scan_ckpt_bytes",
+EXPORTS = ("ssm_version", "ssm_last_error_string", "ssm_last_kernel_path",
+           "ssm_selective_scan_ckpt_bytes",
            "ssm_selective_scan_fwd", "ssm_selective_scan_bwd_scratch_bytes",
            "ssm_selective_scan_bwd", "ssm_device_error_status",
            "ssm_selective_scan_bwd_noalloc", "ssm_selective_state_update",
@@ -70,6 +71,7 @@ def load_library(path: str = LIB_PATH):
     sp = ctypes.POINTER(Shape)
     lib.ssm_version.restype = i
     lib.ssm_last_error_string.restype = ctypes.c_char_p
+    lib.ssm_last_kernel_path.restype = ctypes.c_char_p
     lib.ssm_selective_scan_ckpt_bytes.argtypes = [sp, ctypes.POINTER(sz)]
     lib.ssm_selective_scan_ckpt_bytes.restype = i
     lib.ssm_selective_scan_bwd_scratch_bytes.argtypes = [sp, i, ctypes.POINTER(sz)]
@@ -109,6 +111,12 @@ def load_library(path: str = LIB_PATH):
 
 def last_error() -> str:
     return load_library().ssm_last_error_string().decode()
+
+
+def last_kernel_path() -> str:
+    """Which kernels the last forward or backward call on this thread used
+    ("fwd:tma", "fwd:general", "fwd:chunked", "bwd:tma", "bwd:general")."""
+    return load_library().ssm_last_kernel_path().decode()
 
 
 def device_error_status(stream=None):

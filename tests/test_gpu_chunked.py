@@ -62,6 +62,7 @@ def check_case(case, require_chunked=True):
     out, last, _, nws = _run(dv, w, chunked=True)
     if require_chunked:
         assert nws > 0, "the shape should take the two-level scan"
+        assert ssm_scan.last_kernel_path() == "fwd:chunked"
     chans = slice(0, w.dim, max(1, w.dim // 64))
     sub = subset_channels(inp, chans)
     ref, rlast = oracle.fwd_workload(sub, w.replace(dim=len(range(w.dim)[chans])))

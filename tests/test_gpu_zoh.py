@@ -82,6 +82,9 @@ def test_zoh_backward(case, a_scale, use_ckpt):
                                     dv["z"], dv["delta_bias"], w.softplus, dv["dout"], ckpt=ck,
                                     zoh=True)
     torch.cuda.synchronize()
+    # dstate 16 with at least one channel row per SM takes the TMA backward
+    tma = w.dstate == 16 and w.batch * w.dim >= 148 and (w.seqlen * (2 if w.io_dtype == "bf16" else 4)) % 16 == 0
+    assert ssm_scan.last_kernel_path() == ("bwd:tma" if tma else "bwd:general")
     ref = oracle.bwd(inp["u_f64"], inp["delta_f64"], inp["A_f64"], inp["B_f64"], inp["C_f64"],
                      inp["D_f64"] if w.has_D else None, inp["z_f64"] if w.has_z else None,
                      inp["delta_bias_f64"] if w.has_bias else None, w.softplus,

@@ -24,7 +24,7 @@ def _consts(path, names):
 def test_zoh_series_coefficients_in_arg_units():
     """φ(x) = Σ x^k/(k+1)!, evaluated in arg = x log2(e): the coefficient of
     arg^k is ln(2)^k/(k+1)!; the switch |x| < 0.1 is |arg| < 0.1 log2(e)."""
-    c = _consts("ssm_fwd_tma.cu", ["L1", "L2", "L3", "L4", "L5", "kSmall"])
+    c = _consts("ssm_common.cuh", ["L1", "L2", "L3", "L4", "L5", "kSmall"])
     for k in range(1, 6):
         want = math.log(2.0) ** k / math.factorial(k + 1)
         assert abs(c[f"L{k}"] - want) <= 2e-7 * want, (k, c[f"L{k}"], want)
@@ -34,9 +34,27 @@ def test_zoh_series_coefficients_in_arg_units():
 def test_zoh_series_accuracy_over_its_range():
     """With those coefficients the degree-5 series in arg stays within its
     truncation error (x^6/7! < 3e-10 for |x| < 0.1) of φ over its range."""
-    c = _consts("ssm_fwd_tma.cu", ["L1", "L2", "L3", "L4", "L5", "kSmall"])
+    c = _consts("ssm_common.cuh", ["L1", "L2", "L3", "L4", "L5", "kSmall"])
     arg = np.linspace(-c["kSmall"], c["kSmall"], 2001)
     x = arg * math.log(2.0)
     exact = np.where(x == 0, 1.0, np.expm1(x) / np.where(x == 0, 1.0, x))
     ser = 1 + arg * (c["L1"] + arg * (c["L2"] + arg * (c["L3"] + arg * (c["L4"] + arg * c["L5"]))))
     assert np.max(np.abs(ser - exact) / exact) < 5e-9
+
+
+def test_zoh_psi_series_coefficients_and_accuracy():
+    """ψ(x) = (x e^x - (e^x - 1))/x² = Σ x^k (k+1)/(k+2)!, evaluated in
+    arg = x log2(e): the coefficient of arg^k is ln(2)^k (k+1)/(k+2)!; the
+    degree-4 series stays within its truncation error (below 2e-8) of ψ for
+    |x| < 0.1."""
+    c = _consts("ssm_common.cuh", ["M1", "M2", "M3", "M4", "kSmallPsi"])
+    for k in range(1, 5):
+        want = math.log(2.0) ** k * (k + 1) / math.factorial(k + 2)
+        assert abs(c[f"M{k}"] - want) <= 2e-7 * want, (k, c[f"M{k}"], want)
+    assert abs(c["kSmallPsi"] - 0.1 / math.log(2.0)) <= 1e-7
+    arg = np.linspace(-c["kSmallPsi"], c["kSmallPsi"], 2001)
+    x = arg * math.log(2.0)
+    xs = np.where(x == 0, 1.0, x)
+    exact = np.where(x == 0, 0.5, (x * np.exp(x) - np.expm1(x)) / (xs * xs))
+    ser = 0.5 + arg * (c["M1"] + arg * (c["M2"] + arg * (c["M3"] + arg * c["M4"])))
+    assert np.max(np.abs(ser - exact) / exact) < 5e-8
