@@ -64,6 +64,35 @@ __device__ __forceinline__ float2 softplus_fast2(float2 r) {
     return v;
 }
 
+// log1p(x) for a pair of x in [0, 1] on the FMA pipe: x q(x), with q a
+// degree-8 polynomial fitted to log1p(x)/x on [0, 1] for minimax relative
+// error (Lawson's iteration on a least-squares fit; 2.3e-7 relative when
+// evaluated in fp32 Horner form).  q(0) = 1, so tiny x keep full relative
+// accuracy.
+__device__ __forceinline__ float2 log1p_poly2(float2 x) {
+    constexpr float Q0 = 0.99999994f, Q1 = -0.499994934f, Q2 = 0.333190978f;
+    constexpr float Q3 = -0.248429865f, Q4 = 0.191060171f, Q5 = -0.136632651f;
+    constexpr float Q6 = 0.0782261342f, Q7 = -0.0295053348f, Q8 = 0.00523271505f;
+    float2 q = __ffma2_rn(x, make_float2(Q8, Q8), make_float2(Q7, Q7));
+    q = __ffma2_rn(x, q, make_float2(Q6, Q6));
+    q = __ffma2_rn(x, q, make_float2(Q5, Q5));
+    q = __ffma2_rn(x, q, make_float2(Q4, Q4));
+    q = __ffma2_rn(x, q, make_float2(Q3, Q3));
+    q = __ffma2_rn(x, q, make_float2(Q2, Q2));
+    q = __ffma2_rn(x, q, make_float2(Q1, Q1));
+    q = __ffma2_rn(x, q, make_float2(Q0, Q0));
+    return __fmul2_rn(x, q);
+}
+
+// softplus on a pair with one SFU op per value: softplus(r) = max(r, 0) +
+// log1p(e^-|r|), the exponential by ex2 on the SFU and log1p by
+// log1p_poly2 on the FMA pipe (softplus_fast2 spends two SFU ops per value).
+__device__ __forceinline__ float2 softplus_fast2_1sfu(float2 r) {
+    const float2 na = make_float2(-fabsf(r.x) * SSM_LOG2E, -fabsf(r.y) * SSM_LOG2E);
+    const float2 l = log1p_poly2(make_float2(ex2(na.x), ex2(na.y)));
+    return __fadd2_rn(make_float2(fmaxf(r.x, 0.f), fmaxf(r.y, 0.f)), l);
+}
+
 // SiLU gate z * sigmoid(z) with sigmoid(z) = (1 + tanh(z/2)) / 2 on the
 // hardware tanh (one SFU op; relative error of tanh.approx ~2^-11, below the
 // rounding of a bf16 result).

@@ -55,6 +55,9 @@
 #ifndef SSM_TMA_STEP_MAJOR
 #define SSM_TMA_STEP_MAJOR 1      // recurrence loop ordered step-major (fp32 B/C, Δ·B only)
 #endif
+#ifndef SSM_TMA_SOFTPLUS_1SFU
+#define SSM_TMA_SOFTPLUS_1SFU 1   // softplus with one SFU op (log1p on the FMA pipe)
+#endif
 #ifndef SSM_TMA_SUM_POLY
 #define SSM_TMA_SUM_POLY 1        // quarters of a lane's states with FMA-pipe exponentials in chunk summaries
 #endif
@@ -70,6 +73,7 @@ constexpr int kTmaUnroll = SSM_TMA_UNROLL;
 constexpr int kPolyPairs = SSM_TMA_POLY_PAIRS;
 constexpr bool kStepMajor = SSM_TMA_STEP_MAJOR != 0;
 constexpr int kSumPolyStates = SSM_TMA_SUM_POLY;
+constexpr bool kSoftplus1Sfu = SSM_TMA_SOFTPLUS_1SFU != 0;
 
 constexpr int align128(int x) { return (x + 127) / 128 * 128; }
 
@@ -436,7 +440,7 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
 #pragma unroll
                     for (int k = 0; k < V; k += 2) {
                         const float2 r = __fadd2_rn(make_float2(dr[k], dr[k + 1]), make_float2(bias[i], bias[i]));
-                        float2 d2 = softplus ? softplus_fast2(r) : r;
+                        float2 d2 = softplus ? (kSoftplus1Sfu ? softplus_fast2_1sfu(r) : softplus_fast2(r)) : r;
                         if (!full_tile) {
                             const bool ok0 = irow[i] >= 0 && (t0 + t + v0 + k) < T1;
                             const bool ok1 = irow[i] >= 0 && (t0 + t + v0 + k + 1) < T1;

@@ -75,6 +75,9 @@ CASES = [
     (2, 2049, 16, "f32", False, False, False, True),
     (5, 300, 32, "bf16", True, True, True, True),
     (64, 5120, 16, "bf16", True, True, True, True),
+    (3, 256, 16, "f32", False, False, False, False),
+    (300, 1024, 16, "bf16", True, True, True, True),
+    (1, 128, 16, "bf16", True, False, True, True),
 ]
 
 
@@ -83,6 +86,22 @@ def test_step_matches_oracle(case):
     batch, dim, N, io, z, D, bias, sp = case
     c = make_case(11 + dim, batch, dim, N, io, z, D, bias, sp)
     run_and_check(c, io)
+
+
+def test_repeated_steps_in_place():
+    """Several steps in a row update the state in place consistently: each
+    step's output and state match the oracle stepped from the previous
+    oracle state."""
+    c = make_case(21, 4, 512, 16, "bf16")
+    st64 = c["state64"]
+    for _ in range(3):
+        out = ssm_scan.selective_state_update(c["state"], c["u"], c["delta"], c["A"], c["B"], c["C"],
+                                              c["D"], c["z"], c["bias"], True)
+        torch.cuda.synchronize()
+        ref_out, st64 = oracle.step(st64, c["u64"], c["delta64"], c["A64"], c["B64"], c["C64"],
+                                    c["D64"], c["z64"], c["bias64"], True)
+        assert_close_io(out.double().cpu().numpy(), ref_out, "bf16", "out")
+        assert_close_io(c["state"].double().cpu().numpy(), st64, "f32", "state")
 
 
 def test_step_unaligned_state_uses_scalar_path():

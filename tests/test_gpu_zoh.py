@@ -94,9 +94,10 @@ def test_zoh_backward(case, a_scale, use_ckpt):
         assert_close_grad(to_f64(g[k]), ref[k], k)
 
 
-@pytest.mark.parametrize("N,io", [(16, "bf16"), (4, "f32"), (32, "f32")])
-def test_zoh_step(N, io):
-    c = make_case(41 + N, 3, 300, N, io)
+@pytest.mark.parametrize("N,io,dim", [(16, "bf16", 300), (4, "f32", 300), (32, "f32", 300),
+                                      (16, "bf16", 384), (16, "f32", 256)])
+def test_zoh_step(N, io, dim):
+    c = make_case(41 + N, 3, dim, N, io)
     out = ssm_scan.selective_state_update(c["state"], c["u"], c["delta"], c["A"], c["B"], c["C"],
                                           c["D"], c["z"], c["bias"], True, zoh=True)
     torch.cuda.synchronize()

@@ -58,3 +58,33 @@ def test_zoh_psi_series_coefficients_and_accuracy():
     exact = np.where(x == 0, 0.5, (x * np.exp(x) - np.expm1(x)) / (xs * xs))
     ser = 0.5 + arg * (c["M1"] + arg * (c["M2"] + arg * (c["M3"] + arg * c["M4"])))
     assert np.max(np.abs(ser - exact) / exact) < 5e-8
+
+
+def test_log1p_polynomial_of_the_one_sfu_softplus():
+    """log1p_poly2: x q(x) with q fitted to log1p(x)/x on [0, 1]; evaluated in
+    fp32 Horner form it stays within 3e-7 relative of log1p over [0, 1], and
+    the softplus built on it, max(r, 0) + log1p(e^-|r|), within 4e-7 relative
+    of the exact softplus over r in [-30, 30] (e^-|r| taken exactly here)."""
+    src = open(os.path.join(CSRC, "ssm_common.cuh")).read()
+    q = []
+    for k in range(9):
+        m = re.search(r"Q%d = ([0-9.eE+-]+)f" % k, src)
+        assert m, k
+        q.append(np.float32(float(m.group(1))))
+
+    def poly(x32):
+        acc = np.full_like(x32, q[8])
+        for k in range(7, -1, -1):
+            acc = (acc * x32 + q[k]).astype(np.float32)
+        return (x32 * acc).astype(np.float32)
+
+    x = np.linspace(0.0, 1.0, 100001).astype(np.float32)
+    ref = np.log1p(x.astype(np.float64))
+    got = poly(x).astype(np.float64)
+    rel = np.abs(got - ref) / np.where(ref == 0, 1.0, ref)
+    assert rel.max() < 3e-7, rel.max()
+    r = np.linspace(-30.0, 30.0, 200001)
+    e = np.exp(-np.abs(r)).astype(np.float32)
+    sp = (np.maximum(r, 0.0).astype(np.float32) + poly(e)).astype(np.float64)
+    exact = np.logaddexp(0.0, r)
+    assert (np.abs(sp - exact) / exact).max() < 4e-7
