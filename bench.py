@@ -492,14 +492,17 @@ def run_ours(args, world, rank, local):
     mufu_peak = SM_COUNT_B200 * MUFU_EX2_PER_CLK_PER_SM * sm_max * 1e6
     achieved = ex2 / mean_s
     alg_bytes = algorithmic_bytes(w, 2 if w.io_dtype == "bf16" else 4, backward=fwdbwd)
-    traffic = None
+    # DRAM bytes of one launch of the dominant kernel, from the ncu capture
+    # named beside it (profiles/dram_traffic.txt); None where there is none
+    traffic, traffic_src = None, None
     tp = os.path.join(ROOT, "profiles", "dram_traffic.txt")
-    if os.path.exists(tp) and not fwdbwd and not proj:
+    if os.path.exists(tp) and not fwdbwd and not proj and not chunked and not args.zoh:
         with open(tp) as f:
             for line in f:
                 parts = line.split()
-                if len(parts) == 2 and not line.startswith("#") and parts[0] == "ssm_fwd_" + w.name:
+                if len(parts) >= 2 and not line.startswith("#") and parts[0] == "ssm_fwd_" + w.name:
                     traffic = int(parts[1])
+                    traffic_src = "profiles/" + parts[2] if len(parts) > 2 else "profiles/dram_traffic.txt"
     line = {
         "metric": METRIC, "value": elems_all / t_max, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": max(3, args.warmup),
@@ -514,6 +517,7 @@ def run_ours(args, world, rank, local):
         "gbs": alg_bytes / mean_s / 1e9,
         "roofline": {"bound": "alu", "achieved": achieved / 1e12, "peak": mufu_peak / 1e12,
                      "unit": "Tex2/s", "frac": achieved / mufu_peak, "traffic": traffic,
+                     "traffic_source": traffic_src,
                      "peak_source": f"148 SMs x 16 ex2/clk x {sm_max:.0f} MHz (SFU)",
                      "hbm": {"achieved_gbs": alg_bytes / mean_s / 1e9,
                              "peak_gbs": float(peaks["hbm_gbs"]),
