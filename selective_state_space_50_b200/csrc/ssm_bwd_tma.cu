@@ -46,6 +46,12 @@ namespace ssm {
 namespace {
 
 // Unroll factor of the loop over the 8-step windows of a tile.
+#ifndef SSM_BWD_RECOMPUTE_A
+#define SSM_BWD_RECOMPUTE_A 1       // Δ·B: form Ā again in the sweep too
+#endif
+#ifndef SSM_BWD_RECOMPUTE_A_ZOH
+#define SSM_BWD_RECOMPUTE_A_ZOH 1   // zero-order hold: form Ā again in the sweep
+#endif
 #ifndef SSM_BWD_WIN_UNROLL
 #define SSM_BWD_WIN_UNROLL 1
 #endif
@@ -161,6 +167,9 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                const TmaBwdParams p) {
     using Ly = BwdLayout<T, NWC, STAGES>;
     constexpr int N = Ly::N, NS = Ly::NS, TT = Ly::TT, CPW = Ly::CPW;
+    // the reverse sweep forms Ā again instead of keeping it (frees 32
+    // registers per lane for the zero-order-hold factors)
+    constexpr bool kRecomputeA = ZOH ? SSM_BWD_RECOMPUTE_A_ZOH != 0 : SSM_BWD_RECOMPUTE_A != 0;
     constexpr int WS = Ly::WS, XS = Ly::XS, W = Ly::W;
 
     extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -531,7 +540,7 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                             const float h1 = fmaf(a.y, h0, beta.y);
                             h[j] = h1;
                             const float2 hv = make_float2(h0, h1);
-                            ab2[P][j] = a;
+                            if constexpr (!kRecomputeA) ab2[P][j] = a;
                             ahp2[P][j] = __ffma2_rn(beta, make_float2(-1.f, -1.f), hv);   // Ā_t h_{t-1}
                             y2[pp] = __ffma2_rn(Cp[pp], hv, y2[pp]);
                             xc[pp] = __fmul2_rn(gyp[pp], hv);
@@ -572,9 +581,19 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
 #pragma unroll
                         for (int pp = 1; pp >= 0; --pp) {
                             const int P = 2 * hh + pp;
+                            // Ā of this pair: kept from the recompute, or (with
+                            // zero-order hold, short of registers) formed again,
+                            // bit for bit the same
+                            float2 aP;
+                            if constexpr (kRecomputeA) {
+                                const float2 argA = __fmul2_rn(dtp[pp], A2p[j]);
+                                aP = make_float2(ex2(argA.x), ex2(argA.y));
+                            } else {
+                                aP = ab2[P][j];
+                            }
                             const float2 cg = __fmul2_rn(Cp[pp], gyp[pp]);
                             const float l1 = fmaf(anext[j], lam[j], cg.y);      // λ of the later step
-                            const float l0 = fmaf(ab2[P][j].y, l1, cg.x);       // λ of the earlier step
+                            const float l0 = fmaf(aP.y, l1, cg.x);              // λ of the earlier step
                             const float2 l2 = make_float2(l0, l1);
                             const float2 wv = __fmul2_rn(l2, ahp2[P][j]);
                             sa2[pp] = __ffma2_rn(A2p[j], wv, sa2[pp]);
@@ -582,11 +601,11 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                                 // β = φ Δ B u: dβ/dΔ = Ā B u, dβ/dA = Δ² ψ B u,
                                 // dβ/du = φ Δ B, dβ/dB = φ Δ u
                                 const float2 arg = __fmul2_rn(dtp[pp], A2p[j]);
-                                const float2 phi = zoh_phi2(arg, ab2[P][j], idt[pp], iA2[j]);
-                                const float2 psi = zoh_psi2(arg, ab2[P][j], phi, idt[pp], iA2[j]);
+                                const float2 phi = zoh_phi2(arg, aP, idt[pp], iA2[j]);
+                                const float2 psi = zoh_psi2(arg, aP, phi, idt[pp], iA2[j]);
                                 const float2 lB = __fmul2_rn(l2, Bp[pp]);
                                 sb2[pp] = __ffma2_rn(lB, phi, sb2[pp]);
-                                sq2[pp] = __ffma2_rn(lB, ab2[P][j], sq2[pp]);
+                                sq2[pp] = __ffma2_rn(lB, aP, sq2[pp]);
                                 const float2 w2 = __ffma2_rn(lB, __fmul2_rn(dup[pp], psi), wv);
                                 dA2[j] = __ffma2_rn(dtp[pp], w2, dA2[j]);
                                 xb[pp] = __fmul2_rn(__fmul2_rn(l2, dup[pp]), phi);
@@ -596,7 +615,7 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                                 xb[pp] = __fmul2_rn(l2, dup[pp]);
                             }
                             lam[j] = l0;
-                            anext[j] = ab2[P][j].x;
+                            anext[j] = aP.x;
                         }
                         *reinterpret_cast<float4 *>(myX + (2 * j + hh) * 4) =
                             make_float4(xb[0].x, xb[0].y, xb[1].x, xb[1].y);
