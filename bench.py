@@ -296,13 +296,14 @@ def run_ours(args, world, rank, local):
         grads = {k: torch.empty(dv[src].shape, **f32) for k, src in
                  (("du", "u"), ("ddelta", "u"), ("dz", "u"), ("dA", "A"), ("dB", "B"), ("dC", "C"),
                   ("dD", "D"), ("ddelta_bias", "delta_bias"))}
-        bwd_only = os.environ.get("SSM_BENCH_BWD_ONLY") == "1"
 
-        def fwd():
+        def fwd(mid=None):
             # one training step of the scan: forward keeping checkpoints, backward
-            if not bwd_only:
-                ssm_scan.fwd_raw(shape, dv["u"], dv["delta"], dv["A"], dv["B"], dv["C"], dv["D"],
-                                 dv["z"], dv["delta_bias"], True, out, last, ck, stream, zoh=args.zoh)
+            # (`mid`, an event recorded between the two launches, times the backward)
+            ssm_scan.fwd_raw(shape, dv["u"], dv["delta"], dv["A"], dv["B"], dv["C"], dv["D"],
+                             dv["z"], dv["delta_bias"], True, out, last, ck, stream, zoh=args.zoh)
+            if mid is not None:
+                mid.record(stream)
             ssm_scan.bwd_raw(shape, dv["u"], dv["delta"], dv["A"], dv["B"], dv["C"], dv["D"],
                              dv["z"], dv["delta_bias"], True, dv["dout"], ck, grads["du"],
                              grads["ddelta"], grads["dA"], grads["dB"], grads["dC"], grads["dD"],
@@ -311,9 +312,6 @@ def run_ours(args, world, rank, local):
                 # data parallel: the ranks hold batch rows of one layer, so the
                 # parameter gradients are summed over ranks (NCCL all-reduce)
                 dp.allreduce_param_grads(grads)
-        if bwd_only:   # checkpoints for the timed backward-only steps
-            ssm_scan.fwd_raw(shape, dv["u"], dv["delta"], dv["A"], dv["B"], dv["C"], dv["D"],
-                             dv["z"], dv["delta_bias"], True, out, last, ck, stream, zoh=args.zoh)
     elif args.segments > 1:
         # the sequence cut into S segments, run with the sharded protocol on
         # this one GPU (pass 1 over all segments, combine, pass 2 over 1..S-1)
@@ -387,17 +385,26 @@ def run_ours(args, world, rank, local):
 
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    mids = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)] if fwdbwd else None
     with ClockSampler(local) as clk:
         barrier(world)
         torch.cuda.synchronize()
         for i in range(args.steps):
             flush.zero_()
             starts[i].record(stream)
-            fwd()
+            if fwdbwd:
+                fwd(mids[i])
+            else:
+                fwd()
             ends[i].record(stream)
         torch.cuda.synchronize()
         barrier(world)
     ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    # forward and backward launches of the training step, each on its own
+    kern_ms = None
+    if fwdbwd:
+        kern_ms = {"fwd": sum(s.elapsed_time(m) for s, m in zip(starts, mids)) / args.steps,
+                   "bwd": sum(m.elapsed_time(e) for m, e in zip(mids, ends)) / args.steps}
     t_dev = sum(ms) / 1e3
     t_max = max_over_ranks(t_dev, world)
     elems_all = world * args.steps * w.batch * w.dim * w.seqlen * w.dstate
@@ -519,22 +526,29 @@ def run_ours(args, world, rank, local):
     chunked = not (fwdbwd or proj or args.segments > 1) and nws > 0
     peaks, peak_src = measured_peaks()
     mean_s = t_dev / args.steps
-    # one exponential per (step, state) in the forward, and one more in the
-    # backward (its minimum with checkpoints)
-    ex2 = w.batch * w.dim * w.seqlen * w.dstate * (2 if fwdbwd else 1)
+    # The roofline is the dominant kernel's: the forward scan, or in the
+    # training step the backward (timed on its own between events).  Each
+    # needs one exponential per (step, state): Ā of the recurrence, and in the
+    # backward Ā of the reverse sweep (its minimum with checkpoints).
+    ex2 = w.batch * w.dim * w.seqlen * w.dstate
+    kern_s = kern_ms["bwd"] / 1e3 if fwdbwd else mean_s
     sm_max = float(peaks.get("sm_max_mhz") or 1965.0)
     mufu_peak = SM_COUNT_B200 * MUFU_EX2_PER_CLK_PER_SM * sm_max * 1e6
-    achieved = ex2 / mean_s
+    achieved = ex2 / kern_s
     alg_bytes = algorithmic_bytes(w, 2 if w.io_dtype == "bf16" else 4, backward=fwdbwd)
+    # bytes of the dominant kernel alone (the backward's reads and writes)
+    k_bytes = (alg_bytes - algorithmic_bytes(w, 2 if w.io_dtype == "bf16" else 4)
+               if fwdbwd else alg_bytes)
     # DRAM bytes of one launch of the dominant kernel, from the ncu capture
     # named beside it (profiles/dram_traffic.txt); None where there is none
     traffic, traffic_src = None, None
     tp = os.path.join(ROOT, "profiles", "dram_traffic.txt")
-    if os.path.exists(tp) and not fwdbwd and not proj and not chunked and not args.zoh:
+    key = ("ssm_bwd_" if fwdbwd else "ssm_fwd_") + w.name
+    if os.path.exists(tp) and not proj and not chunked and not args.zoh:
         with open(tp) as f:
             for line in f:
                 parts = line.split()
-                if len(parts) >= 2 and not line.startswith("#") and parts[0] == "ssm_fwd_" + w.name:
+                if len(parts) >= 2 and not line.startswith("#") and parts[0] == key:
                     traffic = int(parts[1])
                     traffic_src = "profiles/" + parts[2] if len(parts) > 2 else "profiles/dram_traffic.txt"
     line = {
@@ -549,14 +563,15 @@ def run_ours(args, world, rank, local):
                                    f"replicas x{world} (independent batches)"),
                    "l2": "flushed between steps (256 MiB write, outside the timed events)"},
         "gbs": alg_bytes / mean_s / 1e9,
-        "roofline": {"bound": "alu", "achieved": achieved / 1e12, "peak": mufu_peak / 1e12,
+        "roofline": {"bound": "alu", "kernel": "backward" if fwdbwd else "forward",
+                     "achieved": achieved / 1e12, "peak": mufu_peak / 1e12,
                      "unit": "Tex2/s", "frac": achieved / mufu_peak, "traffic": traffic,
                      "traffic_source": traffic_src,
                      "peak_source": f"148 SMs x 16 ex2/clk x {sm_max:.0f} MHz (SFU)",
-                     "hbm": {"achieved_gbs": alg_bytes / mean_s / 1e9,
+                     "hbm": {"achieved_gbs": k_bytes / kern_s / 1e9,
                              "peak_gbs": float(peaks["hbm_gbs"]),
-                             "frac": alg_bytes / mean_s / 1e9 / float(peaks["hbm_gbs"]),
-                             "peak_source": peak_src, "alg_bytes": alg_bytes}},
+                             "frac": k_bytes / kern_s / 1e9 / float(peaks["hbm_gbs"]),
+                             "peak_source": peak_src, "alg_bytes": k_bytes}},
         "clocks": clk.summary(),
         "e2e": {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
@@ -568,6 +583,11 @@ def run_ours(args, world, rank, local):
                                       (2 * args.segments if args.segments > 1 else
                                        3 if chunked else 1)),
     }
+    if kern_ms:
+        line["kernels_ms"] = dict(kern_ms, note=(
+            "CUDA events on the launching stream around the forward launch and around the "
+            "backward call (its gradient zero-fills included"
+            + (", and the parameter-gradient all-reduce" if world > 1 else "") + ")"))
     if args.zoh:
         line["config"]["discretization"] = "zero-order hold"
     if chunked:

@@ -66,6 +66,7 @@ struct TmaBwdParams {
     int P, dim, L, n_ckpt;
     int softplus, has_z;
     int rows_max;
+    int vec_out;     // du, ddelta, dz 16-byte aligned and L % 4 == 0
     int *err;
 };
 
@@ -91,7 +92,12 @@ struct BwdLayout {
     static constexpr int WS = TT + 4;                                  // row of wDt / wDu / wGy
     static constexpr int XS = W * NS + 4;                              // row of the transpose
     static constexpr int kWdt = 0, kWdu = CPW * WS, kWgy = 2 * CPW * WS;
-    static constexpr int kWx = 3 * CPW * WS;                           // [32][XS]
+    // per-element sums over the states, written by the windows and read by
+    // the tile's epilogue: y, Σ λ A Ā h (scaled to units of A), Σ λ B, and
+    // with zero-order hold Σ λ B Ā
+    static constexpr int kWy = 3 * CPW * WS, kWsa = 4 * CPW * WS, kWsb = 5 * CPW * WS;
+    static constexpr int kWsq = 6 * CPW * WS;
+    static constexpr int kWx = 7 * CPW * WS;                           // [32][XS]
     static constexpr int WBUF = (kWx + 32 * XS) * 4;
     // dB/dC tile accumulator: [B or C][batch row][state][TT], rows rotated
     static constexpr int DBC_PAR = 2 * 2 * N * TT;
@@ -341,6 +347,8 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
     const int it_rl = lane / (TT / W), it_t = (lane % (TT / W)) * W;   // prep: row, step offset
     float *wbase = reinterpret_cast<float *>(smem + Ly::kW + warp * Ly::WBUF);
     float *wDt = wbase + Ly::kWdt, *wDu = wbase + Ly::kWdu, *wGy = wbase + Ly::kWgy;
+    float *wY = wbase + Ly::kWy, *wSa = wbase + Ly::kWsa, *wSb = wbase + Ly::kWsb;
+    float *wSq = wbase + Ly::kWsq;
     float *wX = wbase + Ly::kWx;
     float *myX = wX + lane * XS;
 
@@ -348,7 +356,7 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
     float2 iA2[NS];                                            // 1 / A twice (zero-order hold)
     float lam[NS], anext[NS];
     float4 hpre = make_float4(0.f, 0.f, 0.f, 0.f);             // checkpoint of the next window
-    float dD_acc = 0.f, db_acc = 0.f, Dd = 0.f, bias_c = 0.f, i_bias = 0.f;
+    float dD_acc = 0.f, db_acc = 0.f, i_D = 0.f, i_bias = 0.f;
     int row = 0, d = 0, bsel = 0, wb = 0, irow = -1;
     bool live = false, straddle = false;
     unsigned b1mask = 0;                                       // channels of the second batch row
@@ -380,11 +388,10 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                 lam[j] = 0.f;
                 anext[j] = 1.f;
             }
-            Dd = (live && p.D) ? p.D[d] : 0.f;
-            bias_c = (live && p.delta_bias) ? p.delta_bias[d] : 0.f;
             const int rr = wrow0 + it_rl;
             irow = rr < q1 ? rr : -1;
             i_bias = (irow >= 0 && p.delta_bias) ? p.delta_bias[rr % p.dim] : 0.f;
+            i_D = (irow >= 0 && p.D) ? p.D[rr % p.dim] : 0.f;
             dD_acc = 0.f;
             db_acc = 0.f;
             // starting state of the first window visited (the one holding step L-1)
@@ -625,33 +632,83 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                     if constexpr (ZOH) sqv[hh] = group_reduce4(sq2[0], sq2[1], g);
                 }
                 reduce_x(0, tw);
-                // per-element results: lane (g, c) finishes steps g and g + 4 of channel c
-                if (live) {
+                // per-element sums of the window for the epilogue: lane (g, c)
+                // holds steps g and g + 4 of channel c (rows of WS floats:
+                // the 32 lanes write 32 different banks)
 #pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int t = g + 4 * e;
-                        if (tgw + t >= p.L) continue;
-                        const int o = c * TT + tw + t;
-                        const float x = IO<T>::to_f(rawU[o]);
-                        const float gv = IO<T>::to_f(rawG[o]);
-                        const float dtv = wDt[c * WS + tw + t], gyv = wGy[c * WS + tw + t];
-                        const float yy = fmaf(Dd, x, yv[e]);
-                        const float sa = sav[e] * 0.69314718f, sb = sbv[e];
-                        const size_t off = (size_t)row * p.L + tgw + t;
-                        if constexpr (HZ) {
-                            const float zz = IO<T>::to_f(rawZ[o]);
-                            const float sg = sigmoid(zz);
-                            __stcs(p.dz + off, gv * yy * sg * fmaf(zz, 1.f - sg, 1.f));
-                        }
-                        const float dDelta = fmaf(x, ZOH ? sqv[e] : sb, sa);
-                        const float ddv = SP ? dDelta * sigmoid(IO<T>::to_f(rawD[o]) + bias_c) : dDelta;
-                        __stcs(p.du + off, fmaf(gyv, Dd, dtv * sb));
-                        __stcs(p.ddelta + off, ddv);
-                        dD_acc = fmaf(gyv, x, dD_acc);
-                        db_acc += ddv;
-                    }
+                for (int e = 0; e < 2; ++e) {
+                    const int o = c * WS + tw + g + 4 * e;
+                    wY[o] = yv[e];
+                    wSa[o] = sav[e] * 0.69314718f;
+                    wSb[o] = sbv[e];
+                    if constexpr (ZOH) wSq[o] = sqv[e];
                 }
                 __syncwarp();   // the transpose buffer is rewritten by the next window
+            }
+            // (3) Epilogue of the tile: lane (it_rl, it_t) finishes steps
+            // it_t .. it_t + 7 of its row (the prep's items): du, dΔ and dz
+            // from the per-element sums, 16-byte loads and streaming stores.
+            if (irow >= 0) {
+                constexpr int V = IO<T>::kVec;
+                float xu[W], xz[W], xd[W], xg[W];
+#pragma unroll
+                for (int v0 = 0; v0 < W; v0 += V) {
+                    const int o = it_rl * TT + it_t + v0;
+                    IO<T>::unpack(*reinterpret_cast<const uint4 *>(rawU + o), xu + v0);
+                    IO<T>::unpack(*reinterpret_cast<const uint4 *>(rawG + o), xg + v0);
+                    if constexpr (SP) IO<T>::unpack(*reinterpret_cast<const uint4 *>(rawD + o), xd + v0);
+                    if constexpr (HZ) IO<T>::unpack(*reinterpret_cast<const uint4 *>(rawZ + o), xz + v0);
+                }
+                const int ro = it_rl * WS + it_t;
+                float rdu[W], rdd[W], rdz[W];
+#pragma unroll
+                for (int e = 0; e < W; e += 4) {
+                    const float4 dt4 = *reinterpret_cast<const float4 *>(wDt + ro + e);
+                    const float4 gy4 = *reinterpret_cast<const float4 *>(wGy + ro + e);
+                    const float4 y4 = *reinterpret_cast<const float4 *>(wY + ro + e);
+                    const float4 sa4 = *reinterpret_cast<const float4 *>(wSa + ro + e);
+                    const float4 sb4 = *reinterpret_cast<const float4 *>(wSb + ro + e);
+                    float4 sq4 = sb4;
+                    if constexpr (ZOH) sq4 = *reinterpret_cast<const float4 *>(wSq + ro + e);
+                    const float dt[4] = {dt4.x, dt4.y, dt4.z, dt4.w}, gy[4] = {gy4.x, gy4.y, gy4.z, gy4.w};
+                    const float yv4[4] = {y4.x, y4.y, y4.z, y4.w}, sa[4] = {sa4.x, sa4.y, sa4.z, sa4.w};
+                    const float sb[4] = {sb4.x, sb4.y, sb4.z, sb4.w}, sq[4] = {sq4.x, sq4.y, sq4.z, sq4.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float x = xu[e + i];
+                        if constexpr (HZ) {
+                            const float zz = xz[e + i], sg = sigmoid(zz);
+                            const float yy = fmaf(i_D, x, yv4[i]);
+                            rdz[e + i] = xg[e + i] * yy * sg * fmaf(zz, 1.f - sg, 1.f);
+                        }
+                        // dΔ: the A term, and u times Σ λ B (Δ·B) or Σ λ B Ā (zero-order hold)
+                        const float dDelta = fmaf(x, sq[i], sa[i]);
+                        rdd[e + i] = SP ? dDelta * sigmoid(xd[e + i] + i_bias) : dDelta;
+                        rdu[e + i] = fmaf(gy[i], i_D, dt[i] * sb[i]);
+                        // prep zeroed gy past the end of the sequence
+                        dD_acc = fmaf(gy[i], x, dD_acc);
+                        if ((t0 + it_t + e + i) < p.L) db_acc += rdd[e + i];
+                    }
+                }
+                const size_t off = (size_t)irow * p.L + t0 + it_t;
+                if (p.vec_out && t0 + it_t + W <= p.L) {
+#pragma unroll
+                    for (int e = 0; e < W; e += 4) {
+                        __stcs(reinterpret_cast<float4 *>(p.du + off + e), make_float4(rdu[e], rdu[e + 1], rdu[e + 2], rdu[e + 3]));
+                        __stcs(reinterpret_cast<float4 *>(p.ddelta + off + e), make_float4(rdd[e], rdd[e + 1], rdd[e + 2], rdd[e + 3]));
+                        if constexpr (HZ)
+                            __stcs(reinterpret_cast<float4 *>(p.dz + off + e), make_float4(rdz[e], rdz[e + 1], rdz[e + 2], rdz[e + 3]));
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < W; ++e) {
+                        if (t0 + it_t + e < p.L) {
+                            __stcs(p.du + off + e, rdu[e]);
+                            __stcs(p.ddelta + off + e, rdd[e]);
+                            if constexpr (HZ) __stcs(p.dz + off + e, rdz[e]);
+                        }
+                    }
+                }
             }
         }
         __syncwarp();
@@ -667,13 +724,13 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                 for (int j = 0; j < NS; ++j) atomicAdd(p.dA + (size_t)d * N + g * NS + j, dA2[j].x + dA2[j].y);
             }
 #pragma unroll
-            for (int m = CPW; m < 32; m <<= 1) {    // lanes c, c+8, c+16, c+24 share channel c
+            for (int m = 1; m < TT / W; m <<= 1) {   // the epilogue's 4 lanes of a row
                 dD_acc += __shfl_xor_sync(0xffffffffu, dD_acc, m);
                 db_acc += __shfl_xor_sync(0xffffffffu, db_acc, m);
             }
-            if (live && g == 0) {
-                if (p.dD) atomicAdd(p.dD + d, dD_acc);
-                if (p.ddelta_bias) atomicAdd(p.ddelta_bias + d, db_acc);
+            if (irow >= 0 && it_t == 0) {
+                if (p.dD) atomicAdd(p.dD + irow % p.dim, dD_acc);
+                if (p.ddelta_bias) atomicAdd(p.ddelta_bias + irow % p.dim, db_acc);
             }
             k = 0;
             ++q;
@@ -705,6 +762,9 @@ cudaError_t launch_bwd_tma_cfg(const BwdParams &bp, int rows_max, cudaStream_t s
     p.dD = bp.dD; p.dz = bp.dz; p.ddelta_bias = bp.ddelta_bias;
     p.P = P; p.dim = bp.dim; p.L = bp.L; p.n_ckpt = bp.n_ckpt;
     p.softplus = bp.softplus; p.has_z = bp.z != nullptr; p.rows_max = rows_max;
+    p.vec_out = bp.L % 4 == 0 && reinterpret_cast<uintptr_t>(bp.du) % 16 == 0 &&
+                reinterpret_cast<uintptr_t>(bp.ddelta) % 16 == 0 &&
+                (!bp.z || reinterpret_cast<uintptr_t>(bp.dz) % 16 == 0);
     p.err = device_error_word();
     if (!p.err) return cudaErrorInvalidDevice;
     auto kern = bwd_tma_kernel<T, NWC, STAGES, HZ, SP, ALN, ZOH>;
