@@ -84,13 +84,19 @@ struct BwdLayout {
     static constexpr int RAW_BC = NPIECE * PIECE;
     static constexpr int kBC0 = bwd_align1024(4 * RAW_CH);
     static constexpr int STAGE = bwd_align1024(kBC0 + 2 * RAW_BC);
-    // B and C of a tile in fp32, [B or C][batch row][state][TT] with swizzled
-    // 16-byte chunks; two buffers (tiles alternate)
-    static constexpr int BCF = 2 * 2 * N * TT;                         // floats per buffer
+    // B and C of a tile in fp32, [B or C][batch row][state][TT]: rows of
+    // BRS floats and a 16-byte pad after the first 8 states of a batch row,
+    // so that the rows a warp reads at once (states 4g + j and, with the
+    // neighbour-channel pairing, 4g + (j ^ 2)) start in 8 different banks;
+    // two buffers (tiles alternate)
+    static constexpr int BRS = TT + 4;
+    static constexpr int BROW = N * BRS + 4;                           // one batch row of B or C
+    static constexpr int BCF = 2 * 2 * BROW;                           // floats per buffer
     static constexpr int W = 8;                                        // window = checkpoint chunk
     static constexpr int NWIN = TT / W;
     static constexpr int WS = TT + 4;                                  // row of wDt / wDu / wGy
     static constexpr int XS = W * NS + 4;                              // row of the transpose
+    static constexpr int XP = W * NS / 2 + 4;                          // the same after the pairing
     static constexpr int kWdt = 0, kWdu = CPW * WS, kWgy = 2 * CPW * WS;
     // per-element sums over the states, written by the windows and read by
     // the tile's epilogue: y, Σ λ A Ā h (scaled to units of A), Σ λ B, and
@@ -111,7 +117,8 @@ struct BwdLayout {
     static_assert(kAlloc <= 227 * 1024, "shared memory budget");
     static_assert(CPW * (TT / W) == 32, "one prep item of 8 steps per lane");
     static_assert(SSM_CKPT_CHUNK == W, "windows are checkpoint chunks");
-    static_assert(WS % 4 == 0 && XS == 36 && TT == 32 && NT == 4 && W == 8, "row shapes");
+    static_assert(WS % 4 == 0 && XS == 36 && XP == 20 && TT == 32 && NT == 4 && W == 8, "row shapes");
+    static_assert(BROW % 4 == 0, "16-byte rows");
 };
 
 // Column of step t of state n in the dB/dC accumulator.  The rotation puts
@@ -119,9 +126,9 @@ struct BwdLayout {
 // into 32 different banks.
 __device__ __forceinline__ int dbc_col(int n, int t) { return (t + 8 * (n >> 2) + (n & 3)) & 31; }
 
-// Physical 16-byte chunk of chunk `ch` in row `row` of the fp32 B/C tile:
-// the four state groups of a warp read different banks.
-__device__ __forceinline__ int bcf_chunk(int row, int ch) { return ch ^ ((row >> 2) & 7); }
+// Offset (floats) of state row n of one batch row in the fp32 B/C tile.
+template <int BRS>
+__device__ __forceinline__ int bcf_row(int n) { return n * BRS + (n >> 3) * 4; }
 
 __device__ __forceinline__ void red_add_v4(float *addr, float4 v) {
     asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(v.x), "f"(v.y),
@@ -136,6 +143,12 @@ __device__ __forceinline__ float4 ldg_f4_now(const float *ptr) {
     asm volatile("ld.global.nc.v4.f32 {%0, %1, %2, %3}, [%4];"
                  : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
                  : "l"(ptr));
+    return v;
+}
+
+__device__ __forceinline__ float2 ldg_f2_now(const float *ptr) {
+    float2 v;
+    asm volatile("ld.global.nc.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "l"(ptr));
     return v;
 }
 
@@ -284,8 +297,8 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                     const float4 f = *reinterpret_cast<const float4 *>(src + rch * 16);
                     v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
                 }
-                float *drow = dstb + (which * 2 * N + rr) * TT;
-                *reinterpret_cast<float4 *>(drow + bcf_chunk(rr, ch) * 4) = make_float4(v[0], v[1], v[2], v[3]);
+                float *drow = dstb + (which * 2 + rr / N) * Ly::BROW + bcf_row<Ly::BRS>(rr % N);
+                *reinterpret_cast<float4 *>(drow + ch * 4) = make_float4(v[0], v[1], v[2], v[3]);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(bcready + (kk & 1));
@@ -344,13 +357,20 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
 
     // ---------------------------------------------------------------- consumers
     const int c = lane % CPW, g = lane / CPW;                 // scan: channel, state group
+    // Pairing of neighbour channels (8-row aligned passes, where a warp's
+    // channels share one batch row): lane c holds state 4g + (j ^ rot) in
+    // register j, so that lanes c and c ^ 1 keep the same two states in
+    // registers 2 and 3 and trade registers 0 and 1 when they sum their dB/dC
+    // partials over the pair.
+    constexpr bool PAIR = ALN;
+    const int rot = PAIR ? (c & 1) << 1 : 0;
     const int it_rl = lane / (TT / W), it_t = (lane % (TT / W)) * W;   // prep: row, step offset
     float *wbase = reinterpret_cast<float *>(smem + Ly::kW + warp * Ly::WBUF);
     float *wDt = wbase + Ly::kWdt, *wDu = wbase + Ly::kWdu, *wGy = wbase + Ly::kWgy;
     float *wY = wbase + Ly::kWy, *wSa = wbase + Ly::kWsa, *wSb = wbase + Ly::kWsb;
     float *wSq = wbase + Ly::kWsq;
     float *wX = wbase + Ly::kWx;
-    float *myX = wX + lane * XS;
+    float *myX = wX + lane * (PAIR ? Ly::XP : XS);
 
     float2 A2p[NS], dA2[NS];                                   // (A log2 e) twice; dA partials
     float2 iA2[NS];                                            // 1 / A twice (zero-order hold)
@@ -360,6 +380,17 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
     int row = 0, d = 0, bsel = 0, wb = 0, irow = -1;
     bool live = false, straddle = false;
     unsigned b1mask = 0;                                       // channels of the second batch row
+    // checkpoint kc of this lane's 4 states, in its register order
+    auto load_ckpt = [&](int kc) -> float4 {
+        if (!(live && kc >= 0)) return make_float4(0.f, 0.f, 0.f, 0.f);
+        const float *b = p.ckpt + ((size_t)row * p.n_ckpt + kc) * N + g * NS;
+        if constexpr (PAIR) {
+            const float2 lo = ldg_f2_now(b + rot), hi = ldg_f2_now(b + (rot ^ 2));
+            return make_float4(lo.x, lo.y, hi.x, hi.y);
+        } else {
+            return ldg_f4_now(b);
+        }
+    };
 
     int s = 0, phase = 0, q = 0, k = 0, q0 = 0, q1 = 0;
     for (int kg = 0; kg < total; ++kg) {
@@ -377,7 +408,7 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
             wb = b1mask != 0 ? 1 : 0;
 #pragma unroll
             for (int j = 0; j < NS; ++j) {
-                const float av = live ? p.A[(size_t)d * N + g * NS + j] : 0.f;
+                const float av = live ? p.A[(size_t)d * N + g * NS + (j ^ rot)] : 0.f;
                 const float a2 = av * SSM_LOG2E;
                 A2p[j] = make_float2(a2, a2);
                 if constexpr (ZOH) {
@@ -396,8 +427,7 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
             db_acc = 0.f;
             // starting state of the first window visited (the one holding step L-1)
             const int kc0 = (p.L - 1) / W - 1;
-            hpre = (live && kc0 >= 0) ? ldg_f4_now(p.ckpt + ((size_t)row * p.n_ckpt + kc0) * N + g * NS)
-                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+            hpre = load_ckpt(kc0);
         }
         const int wrow0 = q0 + warp * CPW;
         {
@@ -450,49 +480,79 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
             }
             __syncwarp();
 
-            const float *bcfB = bcf + (kg & 1) * Ly::BCF + bsel * N * TT;
-            const float *bcfC = bcfB + 2 * N * TT;
-            const int swz = (bsel * 4 + g) & 7;              // bcf_chunk of this lane's rows
+            const float *bcfB = bcf + (kg & 1) * Ly::BCF + bsel * Ly::BROW;
+            const float *bcfC = bcfB + 2 * Ly::BROW;
             auto bc4 = [&](const float *base, int j, int tb) -> float4 {
-                return *reinterpret_cast<const float4 *>(base + (g * NS + j) * TT + (((tb >> 2) ^ swz) << 2));
+                return *reinterpret_cast<const float4 *>(base + bcf_row<Ly::BRS>(g * NS + (j ^ rot)) + tb);
             };
             // Sum of the transpose buffer over the quarter-warp's 8 channels:
             // lane (g, c) takes state 4g + c/2, steps 4(c&1)..4(c&1)+3 of the
             // window, and adds them to accumulator `which` (0: dB, 1: dC).
             auto reduce_x = [&](int which, int tw) {
                 __syncwarp();
-                const float *src = wX + g * CPW * XS + c * 4;
-                const int n = g * NS + (c >> 1), tb = tw + (c & 1) * 4;
+                const int nl = c >> 1, n = g * NS + nl, tb = tw + (c & 1) * 4;
                 float *dst = dbuf + (which * 2 * N + n) * TT;
-                if (ALN || !straddle) {
+                auto add4 = [&](float *row, float4 v) {
+                    atomicAdd(row + dbc_col(n, tb + 0), v.x);
+                    atomicAdd(row + dbc_col(n, tb + 1), v.y);
+                    atomicAdd(row + dbc_col(n, tb + 2), v.z);
+                    atomicAdd(row + dbc_col(n, tb + 3), v.w);
+                };
+                if constexpr (PAIR) {
+                    // after the pairing, state nl of the group is held by the
+                    // lanes of parity 1 (states 0, 1) or 0 (states 2, 3), at
+                    // chunk 2 (half) + (nl & 1) of their rows
+                    const int par = nl < 2 ? 1 : 0;
+                    const float *src = wX + (g * CPW + par) * Ly::XP + ((c & 1) * 2 + (nl & 1)) * 4;
                     float4 s0 = *reinterpret_cast<const float4 *>(src);
 #pragma unroll
-                    for (int cc = 1; cc < CPW; ++cc) s0 = f4add(s0, *reinterpret_cast<const float4 *>(src + cc * XS));
+                    for (int i = 1; i < CPW / 2; ++i)
+                        s0 = f4add(s0, *reinterpret_cast<const float4 *>(src + 2 * i * Ly::XP));
                     __syncwarp();
-                    dst += wb * N * TT;
-                    atomicAdd(dst + dbc_col(n, tb + 0), s0.x);
-                    atomicAdd(dst + dbc_col(n, tb + 1), s0.y);
-                    atomicAdd(dst + dbc_col(n, tb + 2), s0.z);
-                    atomicAdd(dst + dbc_col(n, tb + 3), s0.w);
+                    add4(dst + wb * N * TT, s0);
                 } else {
-                    // channels of two batch rows: one sum per batch row
-                    float4 s0 = make_float4(0.f, 0.f, 0.f, 0.f), s1 = s0;
+                    const float *src = wX + g * CPW * XS + c * 4;
+                    if (!straddle) {
+                        float4 s0 = *reinterpret_cast<const float4 *>(src);
 #pragma unroll
-                    for (int cc = 0; cc < CPW; ++cc) {
-                        const float4 v = *reinterpret_cast<const float4 *>(src + cc * XS);
-                        if ((b1mask >> cc) & 1) s1 = f4add(s1, v);
-                        else s0 = f4add(s0, v);
+                        for (int cc = 1; cc < CPW; ++cc) s0 = f4add(s0, *reinterpret_cast<const float4 *>(src + cc * XS));
+                        __syncwarp();
+                        add4(dst + wb * N * TT, s0);
+                    } else {
+                        // channels of two batch rows: one sum per batch row
+                        float4 s0 = make_float4(0.f, 0.f, 0.f, 0.f), s1 = s0;
+#pragma unroll
+                        for (int cc = 0; cc < CPW; ++cc) {
+                            const float4 v = *reinterpret_cast<const float4 *>(src + cc * XS);
+                            if ((b1mask >> cc) & 1) s1 = f4add(s1, v);
+                            else s0 = f4add(s0, v);
+                        }
+                        __syncwarp();
+                        add4(dst, s0);
+                        add4(dst + N * TT, s1);
                     }
-                    __syncwarp();
-                    atomicAdd(dst + dbc_col(n, tb + 0), s0.x);
-                    atomicAdd(dst + dbc_col(n, tb + 1), s0.y);
-                    atomicAdd(dst + dbc_col(n, tb + 2), s0.z);
-                    atomicAdd(dst + dbc_col(n, tb + 3), s0.w);
-                    dst += N * TT;
-                    atomicAdd(dst + dbc_col(n, tb + 0), s1.x);
-                    atomicAdd(dst + dbc_col(n, tb + 1), s1.y);
-                    atomicAdd(dst + dbc_col(n, tb + 2), s1.z);
-                    atomicAdd(dst + dbc_col(n, tb + 3), s1.w);
+                }
+            };
+            // The dB/dC partials of a half-window (4 states x 4 steps, as
+            // (state, step pair) float2) into this lane's transpose row; with
+            // the pairing, summed with the neighbour channel's first.
+            auto put_x = [&](const float2 (&xv)[NS][2], int hh) {
+                if constexpr (PAIR) {
+#pragma unroll
+                    for (int r = 0; r < 2; ++r) {
+                        float2 o0 = xv[r][0], o1 = xv[r][1];
+                        o0.x = __shfl_xor_sync(0xffffffffu, o0.x, 1);
+                        o0.y = __shfl_xor_sync(0xffffffffu, o0.y, 1);
+                        o1.x = __shfl_xor_sync(0xffffffffu, o1.x, 1);
+                        o1.y = __shfl_xor_sync(0xffffffffu, o1.y, 1);
+                        const float2 k0 = __fadd2_rn(xv[r + 2][0], o0), k1 = __fadd2_rn(xv[r + 2][1], o1);
+                        *reinterpret_cast<float4 *>(myX + (2 * hh + r) * 4) = make_float4(k0.x, k0.y, k1.x, k1.y);
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < NS; ++j)
+                        *reinterpret_cast<float4 *>(myX + (2 * j + hh) * 4) =
+                            make_float4(xv[j][0].x, xv[j][0].y, xv[j][1].x, xv[j][1].y);
                 }
             };
 
@@ -505,8 +565,7 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                 float h[NS] = {hpre.x, hpre.y, hpre.z, hpre.w};
                 {
                     const int kc = tgw / W - 2;             // checkpoint of the next window
-                    hpre = (live && kc >= 0) ? ldg_f4_now(p.ckpt + ((size_t)row * p.n_ckpt + kc) * N + g * NS)
-                                             : make_float4(0.f, 0.f, 0.f, 0.f);
+                    hpre = load_ckpt(kc);
                 }
                 // Forward recompute over pairs of steps (f32x2 arithmetic):
                 // Ā_t, Ā_t h_{t-1}, the y partials and gy h_t (for dC).
@@ -530,12 +589,12 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                             idt[pp] = make_float2(rcp_approx(dtp[pp].x), rcp_approx(dtp[pp].y));
                     }
                     float2 y2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+                    float2 xc[NS][2];                       // gy h (dC partials)
 #pragma unroll
                     for (int j = 0; j < NS; ++j) {
                         const float4 B4 = bc4(bcfB, j, tb), C4 = bc4(bcfC, j, tb);
                         const float2 Bp[2] = {make_float2(B4.x, B4.y), make_float2(B4.z, B4.w)};
                         const float2 Cp[2] = {make_float2(C4.x, C4.y), make_float2(C4.z, C4.w)};
-                        float2 xc[2];
 #pragma unroll
                         for (int pp = 0; pp < 2; ++pp) {
                             const int P = 2 * hh + pp;
@@ -550,11 +609,10 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                             if constexpr (!kRecomputeA) ab2[P][j] = a;
                             ahp2[P][j] = __ffma2_rn(beta, make_float2(-1.f, -1.f), hv);   // Ā_t h_{t-1}
                             y2[pp] = __ffma2_rn(Cp[pp], hv, y2[pp]);
-                            xc[pp] = __fmul2_rn(gyp[pp], hv);
+                            xc[j][pp] = __fmul2_rn(gyp[pp], hv);
                         }
-                        *reinterpret_cast<float4 *>(myX + (2 * j + hh) * 4) =
-                            make_float4(xc[0].x, xc[0].y, xc[1].x, xc[1].y);
                     }
+                    put_x(xc, hh);
                     yv[hh] = group_reduce4(y2[0], y2[1], g);
                 }
                 reduce_x(1, tw);
@@ -579,12 +637,12 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                         for (int pp = 0; pp < 2; ++pp)
                             idt[pp] = make_float2(rcp_approx(dtp[pp].x), rcp_approx(dtp[pp].y));
                     }
+                    float2 xb[NS][2];                       // λ Δu (dB partials)
 #pragma unroll
                     for (int j = 0; j < NS; ++j) {
                         const float4 B4 = bc4(bcfB, j, tb), C4 = bc4(bcfC, j, tb);
                         const float2 Bp[2] = {make_float2(B4.x, B4.y), make_float2(B4.z, B4.w)};
                         const float2 Cp[2] = {make_float2(C4.x, C4.y), make_float2(C4.z, C4.w)};
-                        float2 xb[2];
 #pragma unroll
                         for (int pp = 1; pp >= 0; --pp) {
                             const int P = 2 * hh + pp;
@@ -615,18 +673,17 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                                 sq2[pp] = __ffma2_rn(lB, aP, sq2[pp]);
                                 const float2 w2 = __ffma2_rn(lB, __fmul2_rn(dup[pp], psi), wv);
                                 dA2[j] = __ffma2_rn(dtp[pp], w2, dA2[j]);
-                                xb[pp] = __fmul2_rn(__fmul2_rn(l2, dup[pp]), phi);
+                                xb[j][pp] = __fmul2_rn(__fmul2_rn(l2, dup[pp]), phi);
                             } else {
                                 dA2[j] = __ffma2_rn(dtp[pp], wv, dA2[j]);
                                 sb2[pp] = __ffma2_rn(l2, Bp[pp], sb2[pp]);
-                                xb[pp] = __fmul2_rn(l2, dup[pp]);
+                                xb[j][pp] = __fmul2_rn(l2, dup[pp]);
                             }
                             lam[j] = l0;
                             anext[j] = aP.x;
                         }
-                        *reinterpret_cast<float4 *>(myX + (2 * j + hh) * 4) =
-                            make_float4(xb[0].x, xb[0].y, xb[1].x, xb[1].y);
                     }
+                    put_x(xb, hh);
                     sav[hh] = group_reduce4(sa2[0], sa2[1], g);
                     sbv[hh] = group_reduce4(sb2[0], sb2[1], g);
                     if constexpr (ZOH) sqv[hh] = group_reduce4(sq2[0], sq2[1], g);
@@ -721,7 +778,8 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
             // end of a pass over this CTA's rows: per-channel sums
             if (live) {
 #pragma unroll
-                for (int j = 0; j < NS; ++j) atomicAdd(p.dA + (size_t)d * N + g * NS + j, dA2[j].x + dA2[j].y);
+                for (int j = 0; j < NS; ++j)
+                    atomicAdd(p.dA + (size_t)d * N + g * NS + (j ^ rot), dA2[j].x + dA2[j].y);
             }
 #pragma unroll
             for (int m = 1; m < TT / W; m <<= 1) {   // the epilogue's 4 lanes of a row
