@@ -96,7 +96,10 @@ struct BwdLayout {
     static constexpr int NWIN = TT / W;
     static constexpr int WS = TT + 4;                                  // row of wDt / wDu / wGy
     static constexpr int XS = W * NS + 4;                              // row of the transpose
-    static constexpr int XP = W * NS / 2 + 4;                          // the same after the pairing
+    // the same after the pairing: 16 floats, 16-byte chunk kk of lane 8g + c
+    // stored at chunk kk ^ ((c >> 1) & 3), so that the stores and the
+    // channel-sum reads both meet 8 different banks per quarter-warp
+    static constexpr int XP = W * NS / 2;
     static constexpr int kWdt = 0, kWdu = CPW * WS, kWgy = 2 * CPW * WS;
     // per-element sums over the states, written by the windows and read by
     // the tile's epilogue: y, Σ λ A Ā h (scaled to units of A), Σ λ B, and
@@ -117,7 +120,7 @@ struct BwdLayout {
     static_assert(kAlloc <= 227 * 1024, "shared memory budget");
     static_assert(CPW * (TT / W) == 32, "one prep item of 8 steps per lane");
     static_assert(SSM_CKPT_CHUNK == W, "windows are checkpoint chunks");
-    static_assert(WS % 4 == 0 && XS == 36 && XP == 20 && TT == 32 && NT == 4 && W == 8, "row shapes");
+    static_assert(WS % 4 == 0 && XS == 36 && XP == 16 && TT == 32 && NT == 4 && W == 8, "row shapes");
     static_assert(BROW % 4 == 0, "16-byte rows");
 };
 
@@ -501,13 +504,14 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                 if constexpr (PAIR) {
                     // after the pairing, state nl of the group is held by the
                     // lanes of parity 1 (states 0, 1) or 0 (states 2, 3), at
-                    // chunk 2 (half) + (nl & 1) of their rows
-                    const int par = nl < 2 ? 1 : 0;
-                    const float *src = wX + (g * CPW + par) * Ly::XP + ((c & 1) * 2 + (nl & 1)) * 4;
-                    float4 s0 = *reinterpret_cast<const float4 *>(src);
+                    // chunk 2 (half) + (nl & 1) of their rows; row par + 2i
+                    // stores it at that chunk ^ i
+                    const int par = nl < 2 ? 1 : 0, kk = (c & 1) * 2 + (nl & 1);
+                    const float *src = wX + (g * CPW + par) * Ly::XP;
+                    float4 s0 = *reinterpret_cast<const float4 *>(src + kk * 4);
 #pragma unroll
                     for (int i = 1; i < CPW / 2; ++i)
-                        s0 = f4add(s0, *reinterpret_cast<const float4 *>(src + 2 * i * Ly::XP));
+                        s0 = f4add(s0, *reinterpret_cast<const float4 *>(src + 2 * i * Ly::XP + (kk ^ i) * 4));
                     __syncwarp();
                     add4(dst + wb * N * TT, s0);
                 } else {
@@ -546,7 +550,8 @@ bwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
                         o1.x = __shfl_xor_sync(0xffffffffu, o1.x, 1);
                         o1.y = __shfl_xor_sync(0xffffffffu, o1.y, 1);
                         const float2 k0 = __fadd2_rn(xv[r + 2][0], o0), k1 = __fadd2_rn(xv[r + 2][1], o1);
-                        *reinterpret_cast<float4 *>(myX + (2 * hh + r) * 4) = make_float4(k0.x, k0.y, k1.x, k1.y);
+                        *reinterpret_cast<float4 *>(myX + ((2 * hh + r) ^ ((c >> 1) & 3)) * 4) =
+                            make_float4(k0.x, k0.y, k1.x, k1.y);
                     }
                 } else {
 #pragma unroll
