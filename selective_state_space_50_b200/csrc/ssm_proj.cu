@@ -74,8 +74,9 @@ struct ProjSmem {
     static constexpr int kUsed = kBars + (2 * STAGES + 1) * 8 + 16 + 1024;
     static constexpr int kAlloc = kUsed > 56 * 1024 ? kUsed : 56 * 1024;
     static_assert(kAlloc <= 227 * 1024, "shared memory budget");
-    static_assert(STAGES > 1 || 5 * kAlloc > 228 * 1024, "at most 4 one-stage CTAs per SM");
-    static_assert(STAGES == 1 || 3 * kAlloc > 228 * 1024, "at most 2 deeper-ring CTAs per SM");
+    // CTAs that can share an SM, by shared memory, never need more tensor
+    // memory than its 512 columns (BN each), so no allocation has to wait
+    static_assert((228 * 1024 / kAlloc) * BN <= 512, "tensor-memory columns of co-resident CTAs");
 };
 
 struct ProjSeg {
