@@ -10,9 +10,10 @@
 //
 // The step is memory-bound: the fp32 state (4 N bytes per channel) is read
 // and written once, everything else is a few bytes per channel.  A group of
-// TPC = N / SPT consecutive threads owns one channel, SPT <= 4 states each, so
-// that a warp's state, A, B and C accesses are contiguous 16-byte vectors;
-// the readout is summed over the group with shuffles.
+// TPC = N / SPT consecutive threads owns one channel, SPT <= 8 states each
+// (16-byte vectors, two per thread at SPT = 8), so that a warp's state, A, B
+// and C accesses are contiguous; the readout is summed over the group with
+// shuffles.
 
 #include "ssm_common.cuh"
 #include "ssm_internal.h"
@@ -21,9 +22,11 @@ namespace ssm {
 
 namespace {
 
-// States per thread (at most; a multiple of 4 for vector access).
+// States per thread (at most; a multiple of 4 for vector access).  Eight
+// (two threads per channel at N = 16) measured fastest: 14.8 us against 17.3
+// with four, for 64 x 5120 x 16.
 #ifndef SSM_STEP_SPT
-#define SSM_STEP_SPT 4
+#define SSM_STEP_SPT 8
 #endif
 constexpr int kStepSpt = SSM_STEP_SPT;
 
@@ -49,14 +52,22 @@ __device__ __forceinline__ void load_io(const T *p, float (&f)[SPT]) {
 }
 
 // Channels per thread: all loads of the CPT channels are issued before any
-// arithmetic, so that more memory requests are in flight per thread.
+// arithmetic.  One channel per thread (shorter threads, more of them
+// resident) measured fastest with eight states per thread.
 #ifndef SSM_STEP_CPT
-#define SSM_STEP_CPT 2
+#define SSM_STEP_CPT 1
 #endif
+#ifndef SSM_STEP_BLOCK
+#define SSM_STEP_BLOCK 128
+#endif
+#ifndef SSM_STEP_MIN_BLOCKS
+#define SSM_STEP_MIN_BLOCKS 1
+#endif
+constexpr int kStepBlock = SSM_STEP_BLOCK, kStepMinBlocks = SSM_STEP_MIN_BLOCKS;
 constexpr int kStepCpt = SSM_STEP_CPT;
 
 template <typename T, int N, bool VEC>
-__global__ void __launch_bounds__(256) state_update_kernel(const StepParams p) {
+__global__ void __launch_bounds__(kStepBlock, kStepMinBlocks) state_update_kernel(const StepParams p) {
     constexpr int SPT = N < kStepSpt ? N : kStepSpt;   // states per thread
     constexpr int TPC = N / SPT;           // threads per channel (a power of two)
     constexpr int CPT = kStepCpt;
@@ -136,7 +147,7 @@ template <typename T, int N>
 cudaError_t launch_step_n(const StepParams &p, cudaStream_t stream) {
     constexpr int SPT = N < kStepSpt ? N : kStepSpt;
     constexpr int TPC = N / SPT;
-    const int block = 256;
+    const int block = kStepBlock;
     const long long groups = ((long long)p.dim + kStepCpt - 1) / kStepCpt;
     const long long gx = (groups * TPC + block - 1) / block;
     const long long batch = p.P / p.dim;
