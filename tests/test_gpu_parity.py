@@ -30,10 +30,12 @@ def run_fwd(dv, w, **kw):
     return out, last, ck
 
 
-def check_fwd(w: Workload, channels=None):
+def check_fwd(w: Workload, channels=None, path=None):
     inp = generate(w)
     dv = to_device(inp, w)
     out, last, _ = run_fwd(dv, w)
+    if path is not None:   # the kernel the library chose for this shape
+        assert ssm_scan.last_kernel_path() == path
     if channels is not None:
         sub = subset_channels(inp, channels)
         ref, rlast = oracle.fwd_workload(sub, w)
@@ -54,12 +56,14 @@ def test_fwd_tiny_f32():
 
 @pytest.mark.parametrize("name", ["mamba130m_layer", "mamba2p8b_layer"])
 def test_fwd_layer_shapes_full(name):
-    check_fwd(WORKLOADS[name])
+    check_fwd(WORKLOADS[name], path="fwd:tma")
 
 
 def test_fwd_long_context_sampled_channels():
+    """Through the public forward, which gives the library its workspace: at
+    1 x 2048 channels over 131072 steps it takes the two-level scan."""
     w = WORKLOADS["long_context"]
-    check_fwd(w, channels=slice(0, w.dim, 97))
+    check_fwd(w, channels=slice(0, w.dim, 97), path="fwd:chunked")
 
 
 SMALL = [
@@ -150,7 +154,7 @@ def test_fwd_repeatable_bitwise():
 
 # ------------------------------------------------------------------ backward
 
-def check_bwd(w: Workload, use_ckpt: bool):
+def check_bwd(w: Workload, use_ckpt: bool, path=None):
     inp = generate(w, with_dout=True)
     dv = to_device(inp, w)
     ck = None
@@ -159,6 +163,8 @@ def check_bwd(w: Workload, use_ckpt: bool):
     g = ssm_scan.selective_scan_bwd(dv["u"], dv["delta"], dv["A"], dv["B"], dv["C"], dv["D"],
                                     dv["z"], dv["delta_bias"], w.softplus, dv["dout"], ckpt=ck)
     torch.cuda.synchronize()
+    if path is not None:   # the kernel the library chose for this shape
+        assert ssm_scan.last_kernel_path() == path
     ref = oracle.bwd_workload(inp, w)
     assert set(g) == set(ref)
     errs = {}
@@ -185,7 +191,7 @@ def test_bwd_small(case, use_ckpt):
 
 
 def test_bwd_layer_shape_full():
-    check_bwd(WORKLOADS["mamba130m_layer_fwdbwd"], use_ckpt=True)
+    check_bwd(WORKLOADS["mamba130m_layer_fwdbwd"], use_ckpt=True, path="bwd:tma")
 
 
 # Shapes with dstate 16, 16-byte aligned rows and at least one channel row per
