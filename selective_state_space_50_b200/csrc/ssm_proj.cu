@@ -64,15 +64,18 @@ struct ProjTile {
 };
 
 // Shared memory of a STAGES-deep ring: the ring, then the barriers and the
-// tensor-memory address.  A one-stage kernel asks for at least 56 KB so that
-// at most four CTAs share an SM: four 128-column accumulators fill its 512
-// tensor-memory columns, and no allocation has to wait.  Deeper rings fit at
-// most two (3 stages) or one (6 stages) CTA per SM.
+// tensor-memory address.  A kernel asks for at least a 512/BN share of the
+// SM's 228 KB (less the 1 KB the SM keeps per CTA), so that at most 512/BN
+// CTAs share an SM: their BN-column accumulators fill its 512 tensor-memory
+// columns, and no allocation has to wait (one-stage 128-column tiles: 56 KB,
+// four CTAs; 64-column tiles: eight).  Deeper rings fit at most two (3
+// stages) or one (6 stages) 128-column CTA per SM.
 template <int STAGES, int BN>
 struct ProjSmem {
     static constexpr int kBars = STAGES * ProjTile<BN>::kStage;
     static constexpr int kUsed = kBars + (2 * STAGES + 1) * 8 + 16 + 1024;
-    static constexpr int kAlloc = kUsed > 56 * 1024 ? kUsed : 56 * 1024;
+    static constexpr int kMin = 228 * 1024 / (512 / BN) - 1024;
+    static constexpr int kAlloc = kUsed > kMin ? kUsed : kMin;
     static_assert(kAlloc <= 227 * 1024, "shared memory budget");
     // CTAs that can share an SM, by shared memory, never need more tensor
     // memory than its 512 columns (BN each), so no allocation has to wait
@@ -88,8 +91,14 @@ struct ProjParams {
     ProjSeg seg[3];
     int nseg;
     int M, K, L;
+    int tma_out;    // one output (seg[0] is the whole product): TMA stores through mO
     int *err;
 };
+
+// TMA-store epilogue: each warp stages 32 rows x 64 columns of bf16 (128-byte
+// rows, 16-byte chunks XOR-swizzled by row as the tensor map's 128B swizzle
+// expects) and one lane stores the box.
+constexpr int kOutStg = 32 * 128;
 
 // ------------------------------------------------------------ tcgen05 helpers
 
@@ -158,7 +167,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(uint32_t lo, uint32_t hi) {
 template <int kStages, int kBN>
 __global__ void __launch_bounds__(kThreads, 1)
 proj_gemm_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mB,
-                 const ProjParams p) {
+                 const __grid_constant__ CUtensorMap mO, const ProjParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
     using Tile = ProjTile<kBN>;
@@ -240,7 +249,40 @@ proj_gemm_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__
     // staging rows, then the warp writes 4 rows x 128 bytes per instruction.
     const bool ok = __all_sync(0xffffffffu, mbar_wait(accum, 0, p.err));
     tc_fence_after();
-    if (ok) {
+    if (ok && p.tma_out) {
+        static_assert(4 * kOutStg <= kStage && kOutStg % 1024 == 0, "output staging fits one stage");
+        uint8_t *stg = smem + warp * kOutStg;            // 1024-byte aligned: the swizzle atom
+        const int m = m0 + warp * 32;
+#pragma unroll 1
+        for (int h = 0; h < kBN / 64; ++h) {
+            if (h > 0) {                                 // the previous box has left the staging
+                if (lane == 0) bulk_wait_group_read<0>();
+                __syncwarp();
+            }
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t r[16];
+                tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(h * 64 + c * 16), r);
+                uint4 v0, v1;
+                v0.x = pack_bf16x2(r[0], r[1]);   v0.y = pack_bf16x2(r[2], r[3]);
+                v0.z = pack_bf16x2(r[4], r[5]);   v0.w = pack_bf16x2(r[6], r[7]);
+                v1.x = pack_bf16x2(r[8], r[9]);   v1.y = pack_bf16x2(r[10], r[11]);
+                v1.z = pack_bf16x2(r[12], r[13]); v1.w = pack_bf16x2(r[14], r[15]);
+                uint8_t *row = stg + lane * 128;
+                *reinterpret_cast<uint4 *>(row + (((2 * c) ^ (lane & 7)) << 4)) = v0;
+                *reinterpret_cast<uint4 *>(row + (((2 * c + 1) ^ (lane & 7)) << 4)) = v1;
+            }
+            fence_proxy_async();                          // the staging, seen by the TMA unit
+            __syncwarp();
+            const int n = n0 + h * 64;
+            if (lane == 0 && n < p.L && m < p.M) {
+                tma_store_3d(&mO, stg, n, m, b);
+                bulk_commit_group();
+            }
+        }
+        if (lane == 0) bulk_wait_group<0>();              // stores done before the CTA leaves
+        __syncwarp();
+    } else if (ok) {
         __nv_bfloat16 *stg = reinterpret_cast<__nv_bfloat16 *>(smem + warp * kStgWarp);
         const int srow = lane / 8, schunk = lane % 8;     // write-out: row within 4, 16-byte chunk
 #pragma unroll 1
@@ -283,8 +325,8 @@ proj_gemm_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__
 }
 
 template <int STAGES, int BN>
-cudaError_t launch_proj_gemm(const CUtensorMap &mA, const CUtensorMap &mB, const ProjParams &p, int batch,
-                             cudaStream_t stream) {
+cudaError_t launch_proj_gemm(const CUtensorMap &mA, const CUtensorMap &mB, const CUtensorMap &mO,
+                             const ProjParams &p, int batch, cudaStream_t stream) {
     constexpr int smem = ProjSmem<STAGES, BN>::kAlloc;
     static bool attr_done = false;
     if (!attr_done) {
@@ -293,9 +335,19 @@ cudaError_t launch_proj_gemm(const CUtensorMap &mA, const CUtensorMap &mB, const
         attr_done = true;
     }
     const dim3 grid((unsigned)((p.L + BN - 1) / BN), (unsigned)((p.M + kBM - 1) / kBM), (unsigned)batch);
-    proj_gemm_kernel<STAGES, BN><<<grid, kThreads, smem, stream>>>(mA, mB, p);
+    proj_gemm_kernel<STAGES, BN><<<grid, kThreads, smem, stream>>>(mA, mB, mO, p);
     return cudaGetLastError();
 }
+
+// dt_proj's output through TMA stores (1) or the row-store epilogue (0).
+#ifndef SSM_PROJ_TMA_STORE
+#define SSM_PROJ_TMA_STORE 1
+#endif
+
+// Tile width of the one-slice contraction (dt_proj at rank <= 64).
+#ifndef SSM_PROJ_SHORT_BN
+#define SSM_PROJ_SHORT_BN 128
+#endif
 
 // Ring depth and tile width of the long contraction (x_proj).
 #ifndef SSM_PROJ_LONG_STAGES
@@ -310,12 +362,12 @@ cudaError_t launch_proj_gemm(const CUtensorMap &mA, const CUtensorMap &mB, const
 // MMAs and stores.  Two or three slices (larger ranks): the whole contraction
 // in flight at once, two CTAs per SM.  Longer (x_proj streams the
 // activations): a 6-stage ring.
-cudaError_t launch_proj_any(const CUtensorMap &mA, const CUtensorMap &mB, const ProjParams &p, int batch,
-                            cudaStream_t stream) {
+cudaError_t launch_proj_any(const CUtensorMap &mA, const CUtensorMap &mB, const CUtensorMap &mO,
+                            const ProjParams &p, int batch, cudaStream_t stream) {
     const int nk = (p.K + kBK - 1) / kBK;
-    if (nk <= 1) return launch_proj_gemm<1, 128>(mA, mB, p, batch, stream);
-    if (nk <= 3) return launch_proj_gemm<3, 128>(mA, mB, p, batch, stream);
-    return launch_proj_gemm<SSM_PROJ_LONG_STAGES, SSM_PROJ_LONG_BN>(mA, mB, p, batch, stream);
+    if (nk <= 1) return launch_proj_gemm<1, SSM_PROJ_SHORT_BN>(mA, mB, mO, p, batch, stream);
+    if (nk <= 3) return launch_proj_gemm<3, 128>(mA, mB, mO, p, batch, stream);
+    return launch_proj_gemm<SSM_PROJ_LONG_STAGES, SSM_PROJ_LONG_BN>(mA, mB, mO, p, batch, stream);
 }
 
 }  // namespace
@@ -337,17 +389,23 @@ cudaError_t launch_projections(const ProjShape &s, const void *x, const void *W_
     p.seg[2] = {C, R + N, N};
     p.nseg = 3;
     p.M = M1; p.K = s.dim; p.L = s.seqlen; p.err = err;
-    cudaError_t e = launch_proj_any(mA, mB, p, s.batch, stream);
+    p.tma_out = 0;   // three outputs (dt_low, B, C): the row-store epilogue
+    cudaError_t e = launch_proj_any(mA, mB, mA, p, s.batch, stream);
     if (e != cudaSuccess) return e;
     // dt_proj: A = W_dt [D x R], Bm = dt_low [batch][R][L]
     if (!make_tma_map_2d(&mA, W_dt, true, (uint64_t)s.dim, (uint64_t)R, kBK, kBM, true) ||
         !make_tma_map_bf16_3d(&mB, dt_low, (uint64_t)s.seqlen, (uint64_t)R, (uint64_t)s.batch, 64, kBK))
         return cudaErrorInvalidValue;
+    // delta [batch][D][L] written by TMA stores of 64-column x 32-row boxes
+    CUtensorMap mO;
+    if (!make_tma_map_bf16_3d(&mO, delta, (uint64_t)s.seqlen, (uint64_t)s.dim, (uint64_t)s.batch, 64, 32))
+        return cudaErrorInvalidValue;
     ProjParams q{};
     q.seg[0] = {delta, 0, s.dim};
     q.nseg = 1;
     q.M = s.dim; q.K = R; q.L = s.seqlen; q.err = err;
-    return launch_proj_any(mA, mB, q, s.batch, stream);
+    q.tma_out = SSM_PROJ_TMA_STORE;
+    return launch_proj_any(mA, mB, mO, q, s.batch, stream);
 }
 
 }  // namespace ssm
