@@ -48,6 +48,18 @@ def measured_peaks():
     return {"hbm_gbs": FALLBACK_HBM_GBS, "sm_max_mhz": 1965.0}, "fallback"
 
 
+def kernel_source_matches(tag):
+    """tag = "<file>@<sha1 prefix>": the kernel source a DRAM-traffic capture
+    was taken with; True while csrc/<file> still has that hash."""
+    import hashlib
+    name, _, digest = tag.partition("@")
+    path = os.path.join(ROOT, "selective_state_space_50_b200", "csrc", name)
+    if not digest or not os.path.exists(path):
+        return False
+    with open(path, "rb") as f:
+        return hashlib.sha1(f.read()).hexdigest().startswith(digest)
+
+
 def algorithmic_bytes(w, io_bytes, with_last_state=True, backward=False):
     """HBM bytes a fused forward must move (and, with backward, the backward
     too): every input read once, every output written once."""
@@ -551,6 +563,9 @@ def run_ours(args, world, rank, local):
                 if len(parts) >= 2 and not line.startswith("#") and parts[0] == key:
                     traffic = int(parts[1])
                     traffic_src = "profiles/" + parts[2] if len(parts) > 2 else "profiles/dram_traffic.txt"
+                    if len(parts) > 3 and not kernel_source_matches(parts[3]):
+                        traffic = None
+                        traffic_src += " (stale: " + parts[3].split("@")[0] + " changed since the capture)"
     line = {
         "metric": METRIC, "value": elems_all / t_max, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": max(3, args.warmup),
