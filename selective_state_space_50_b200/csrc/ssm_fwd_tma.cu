@@ -49,6 +49,9 @@
 #ifndef SSM_TMA_F32BC
 #define SSM_TMA_F32BC 1       // producer rewrites B/C as fp32 (32-step tiles)
 #endif
+#ifndef SSM_TMA_CONV_SUBPART3
+#define SSM_TMA_CONV_SUBPART3 1   // the B/C converter warp on SM sub-partition 3
+#endif
 #ifndef SSM_TMA_WAIT_SUSPEND
 #define SSM_TMA_WAIT_SUSPEND 0    // waits suspend in the barrier unit instead of polling
 #endif
@@ -130,8 +133,13 @@ struct TmaLayout {
     static constexpr int kBar = kW + NWC * WBUF;
     static constexpr int kTotal = kBar + 3 * STAGES * 8;
     static constexpr int kAlloc = kTotal + 1024;   // room to align the base to 1024 B
-    // consumer warps, the TMA warp and (with the fp32 B/C copy) a converter warp
-    static constexpr int kThreads = (NWC + 1 + (F32BC ? 1 : 0)) * 32;
+    // Consumer warps 0..NWC-1, the TMA warp NWC and (with the fp32 B/C copy) a
+    // converter warp.  Warp w runs on SM sub-partition w % 4, and the consumers
+    // fill sub-partitions 0, 1, 2 first, so the converter takes the first index
+    // after the TMA warp on sub-partition 3 (indices between stay idle).
+    static constexpr int kConvWarp =
+        SSM_TMA_CONV_SUBPART3 ? NWC + 1 + (3 - (NWC + 1) % 4 + 4) % 4 : NWC + 1;
+    static constexpr int kThreads = (F32BC ? kConvWarp + 1 : NWC + 1) * 32;
     static constexpr int CHUNK = 8;                            // steps per prep/epilogue item
     static constexpr int ITEMS = CPW * (TT / CHUNK);           // (row, chunk) items per warp
     static_assert(kAlloc <= 227 * 1024, "shared memory budget");
@@ -292,8 +300,9 @@ fwd_tma_kernel(const __grid_constant__ CUtensorMap m_delta, const __grid_constan
             if (!mbar_wait(full + (kk % STAGES), (kk / STAGES) & 1, p.err)) break;
         return;
     }
+    if (warp > NWC && warp != Ly::kConvWarp) return;   // idle slots before the converter
     if constexpr (Ly::F32BC) {
-        if (warp == NWC + 1) {
+        if (warp == Ly::kConvWarp) {
             // ------------------------------------------------ B/C converter
             // Each tile's B and C, once landed, rewritten as fp32 rows in the
             // stage's fp32 area (16-byte chunks swizzled by row / NS), then
