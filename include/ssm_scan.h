@@ -117,6 +117,13 @@ const char *ssm_last_kernel_path(void);
 ssm_status_t ssm_selective_scan_ckpt_bytes(const ssm_shape_t *shape, size_t *bytes);
 
 /*
+ * The same size under the name of the boundary's original plan: the bytes
+ * of the checkpoint buffer (the backward's workspace when the caller keeps
+ * the forward's checkpoints).  Identical to ssm_selective_scan_ckpt_bytes.
+ */
+ssm_status_t ssm_selective_scan_workspace_size(const ssm_shape_t *shape, size_t *ckpt_bytes);
+
+/*
  * Forward selective scan (see the header comment for the arithmetic).
  *
  *  u, delta, A, B, C : required inputs.
@@ -329,6 +336,10 @@ ssm_status_t ssm_selective_state_update_ex(const ssm_shape_t *shape, const ssm_o
  * instead of hanging the stream.
  */
 ssm_status_t ssm_device_error_status(void *stream);
+
+/* The same check under the name of the boundary's original plan; identical
+ * to ssm_device_error_status. */
+ssm_status_t ssm_check_device_errors(void *stream);
 
 /*
  * Diagnostic: launches on `stream` a one-warp kernel whose bounded wait (on a

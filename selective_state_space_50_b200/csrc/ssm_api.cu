@@ -152,6 +152,10 @@ ssm_status_t ssm_selective_scan_ckpt_bytes(const ssm_shape_t *shape, size_t *byt
     return ok();
 }
 
+ssm_status_t ssm_selective_scan_workspace_size(const ssm_shape_t *shape, size_t *ckpt_bytes) {
+    return ssm_selective_scan_ckpt_bytes(shape, ckpt_bytes);
+}
+
 ssm_status_t ssm_selective_scan_bwd_scratch_bytes(const ssm_shape_t *shape, int have_ckpt,
                                                   size_t *bytes) {
     SSM_TRY(check_shape(shape));
@@ -489,5 +493,7 @@ ssm_status_t ssm_device_error_status(void *stream) {
     if (v) return fail(SSM_ERR_TIMEOUT, "a bounded wait inside a kernel gave up (code %d)", v);
     return ok();
 }
+
+ssm_status_t ssm_check_device_errors(void *stream) { return ssm_device_error_status(stream); }
 
 }  // extern "C"

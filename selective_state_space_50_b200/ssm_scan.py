@@ -31,7 +31,8 @@ EXPORTS = ("ssm_version", "ssm_last_error_string", "ssm_last_kernel_path",
            "ssm_selective_state_update_ex", "ssm_selftest_wait_timeout",
            "ssm_selection_projections", "ssm_selective_scan_fwd_segment",
            "ssm_scan_combine_carries", "ssm_selective_scan_fwd_workspace_bytes",
-           "ssm_selective_scan_fwd_ws")
+           "ssm_selective_scan_fwd_ws", "ssm_selective_scan_workspace_size",
+           "ssm_check_device_errors")
 SSM_DISC_DELTA_B, SSM_DISC_ZOH = 0, 1
 NOALLOC_SCRATCH_BYTES = 32 << 20  # SSM_NOALLOC_SCRATCH_BYTES in include/ssm_scan.h
 
@@ -82,6 +83,10 @@ def load_library(path: str = LIB_PATH):
     lib.ssm_selective_scan_bwd.restype = i
     lib.ssm_device_error_status.argtypes = [vp]
     lib.ssm_device_error_status.restype = i
+    lib.ssm_selective_scan_workspace_size.argtypes = [sp, ctypes.POINTER(sz)]
+    lib.ssm_selective_scan_workspace_size.restype = i
+    lib.ssm_check_device_errors.argtypes = [vp]
+    lib.ssm_check_device_errors.restype = i
     lib.ssm_selective_scan_bwd_noalloc.argtypes = [sp] + [vp] * 8 + [i] + [vp] * 10
     lib.ssm_selective_scan_bwd_noalloc.restype = i
     lib.ssm_selective_state_update.argtypes = [sp] + [vp] * 9 + [i] + [vp] * 2

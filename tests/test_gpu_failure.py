@@ -30,3 +30,14 @@ def test_wait_timeout_is_reported_then_cleared_and_the_context_survives():
     # the context is still usable: a forward on the TMA path matches the oracle
     check_fwd(small_workload(2, 2400, 72, 16, "bf16", True, True, True, True, "neg_lognormal"))
     ssm_scan.device_error_status()
+
+
+def test_planned_name_reports_the_same_timeout():
+    """ssm_check_device_errors (the boundary's planned name) reports and clears
+    the word exactly as ssm_device_error_status does."""
+    lib = ssm_scan.load_library()
+    stream = ssm_scan._stream_ptr(None)
+    assert lib.ssm_check_device_errors(stream) == ssm_scan.SSM_OK
+    assert lib.ssm_selftest_wait_timeout(stream) == ssm_scan.SSM_OK
+    assert lib.ssm_check_device_errors(stream) == ssm_scan.SSM_ERR_TIMEOUT
+    assert lib.ssm_check_device_errors(stream) == ssm_scan.SSM_OK
